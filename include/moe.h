@@ -1,0 +1,192 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) library for the LongCat-Flash MoE layer with
+ * zero-computation experts.
+ *
+ * What the layer computes ("衝上熱搜！美團大模型，靠「快」火了", section 零計算專家): the expert
+ * pool holds N SwiGLU FFN experts and Z zero-computation experts (E = N + Z).  A softmax router
+ * R scores all E experts for each token x_t; a per-expert bias b_i is added to the router
+ * probability for the top-K selection only; the gate g_i is the (unbiased, not renormalised)
+ * probability; the output is y_t = sum over the K selected experts of g_i * E_i(x_t), where an
+ * FFN expert is E(x) = W_d (silu(W_g x) * (W_u x)) and a zero expert returns x_t unchanged.
+ * A PID controller on the biases (same page, last paragraph of that section) holds the mean
+ * number of FFN experts per token near a set-point.
+ *
+ * Conventions shared by every entry point
+ *   - All pointers are DEVICE pointers unless stated otherwise; the caller owns every buffer.
+ *     The library never allocates or frees device memory and keeps no per-call state.
+ *   - `stream` is a cudaStream_t passed as void*; every call only enqueues work on it and
+ *     returns without synchronising (except moe_last_device_error).  Calls on one stream are
+ *     ordered; calls sharing a workspace must not run concurrently on different streams.
+ *   - bf16 tensors are arrays of uint16_t bit patterns (moe_bf16).  Layouts are row-major and
+ *     contiguous.  Shapes use the dims struct: T tokens, d model width, N FFN experts of
+ *     intermediate width I, Z zero experts, K experts per token.
+ *   - Limits: T >= 0; d and I positive multiples of 64; N >= 0, Z >= 0, 1 <= N + Z <= 1024;
+ *     1 <= K <= min(N + Z, 32); T * K < 2^31.  Violations return MOE_ERR_SHAPE.
+ *   - Every tensor pointer must be 16-byte aligned (MOE_ERR_ALIGN otherwise); a workspace
+ *     must be 256-byte aligned.  A NULL required pointer returns MOE_ERR_ARG.
+ *   - Errors are reported by the return code before anything is enqueued; a launch failure
+ *     returns MOE_ERR_CUDA.  Kernels never trap: a device-side check that fails (a bounded wait
+ *     that gave up, an expert id or row index out of range) records a code in the workspace's
+ *     status word, skips the offending access and lets the kernel finish; read it with
+ *     moe_last_device_error.  No call aborts the process.
+ *   - T == 0 is valid: outputs are left as described per call (counts zeroed where written),
+ *     and every token-sized pointer (x, y, top-K, dispatch and grouped-row buffers) may then be
+ *     NULL.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t moe_bf16; /* bf16 bit pattern */
+
+typedef struct {
+    int32_t T; /* tokens in the batch */
+    int32_t d; /* model width */
+    int32_t N; /* FFN experts (ids 0 .. N-1) */
+    int32_t Z; /* zero-computation experts (ids N .. N+Z-1) */
+    int32_t K; /* experts selected per token */
+    int32_t I; /* intermediate width of each SwiGLU FFN expert */
+} moe_dims;
+
+/* PID gains and set-point: target = desired mean number of FFN experts per token. */
+typedef struct {
+    float target;
+    float kp;
+    float ki;
+    float kd;
+} moe_pid_params;
+
+enum {
+    MOE_OK = 0,
+    MOE_ERR_ARG = 1,       /* NULL pointer or invalid parameter value */
+    MOE_ERR_SHAPE = 2,     /* dims outside the supported limits */
+    MOE_ERR_ALIGN = 3,     /* pointer not 16-byte (tensor) / 256-byte (workspace) aligned */
+    MOE_ERR_WORKSPACE = 4, /* ws_bytes smaller than required */
+    MOE_ERR_CUDA = 5,      /* a CUDA runtime call or kernel launch failed */
+    MOE_ERR_DEVICE = 6,    /* a device-side check failed (see moe_last_device_error) */
+    MOE_ERR_ARCH = 7       /* the current device is not sm_100 (B200-class) */
+};
+
+/* Device-side status codes reported by moe_last_device_error (0 = none). */
+enum {
+    MOE_DEV_OK = 0,
+    MOE_DEV_WAIT_TIMEOUT = 0x100, /* a pipeline wait in the grouped GEMM gave up (bounded) */
+    MOE_DEV_BAD_EXPERT = 0x200,   /* an expert id outside [0, N+Z) was met */
+    MOE_DEV_BAD_ROWS = 0x300      /* group offsets not monotone or beyond T*K rows */
+};
+
+/* Human-readable text for a return code (host only; never NULL). */
+const char *moe_strerror(int code);
+
+/* Workspace bytes needed by moe_forward for these dims (0 for invalid dims).  The workspace
+ * holds the status word, router logits, top-K results, dispatch tables, the grouped
+ * activations x_perm [T*K, d], the SwiGLU activations h [T*K, I] and the expert outputs
+ * y_perm [T*K, d]; about (2d + I) * 2 * T * K bytes plus small tables. */
+size_t moe_workspace_size(const moe_dims *dims);
+
+/* Scratch bytes needed by the staged calls (moe_route, moe_dispatch, moe_expert_ffn): the
+ * status word, split-K router logits and per-chunk histograms.  Always <= the above. */
+size_t moe_scratch_size(const moe_dims *dims);
+
+/* Router R and biased top-K ("衝上熱搜！美團大模型，靠「快」火了", §零計算專家: softmax
+ * router over all N+Z experts; b_i shifts the selection score only).
+ *   x        [T, d] bf16            tokens
+ *   W_r      [N+Z, d] bf16          router weights; logits l = x W_r^T (fp32 accumulation on
+ *                                   tensor cores)
+ *   b        [N+Z] fp32             per-expert selection bias
+ *   topk_idx [T, K] int32   (out)   selected expert ids, ascending
+ *   topk_gate[T, K] fp32    (out)   g_i = softmax(l)_i of the selected ids (not renormalised)
+ *   gap      [T] fp32       (out, nullable)  s_(K) - s_(K+1) with s = softmax(l) + b
+ *                                   (+inf when K == N+Z); a small gap marks a near-tie
+ * Exact score ties go to the lower expert id. */
+int moe_route(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *W_r, const float *b,
+              int32_t *topk_idx, float *topk_gate, float *gap, void *ws, size_t ws_bytes,
+              void *stream);
+
+/* Dispatch: group the FFN slots by expert (zero-expert slots are never copied).  Stable
+ * counting sort with key (expert id, token), deterministic.
+ *   x         [T, d] bf16, topk_idx/topk_gate [T, K] as produced by moe_route (ids in
+ *             ascending order per token, each in [0, N+Z))
+ *   counts    [N+Z] int32   (out)   slots per expert (zero experts included)
+ *   offsets   [N+1] int32   (out)   row offset of each FFN expert's group; offsets[N] = A,
+ *                                   the number of FFN slots
+ *   perm_tok  [T*K] int32   (out)   token of grouped row r (r < A)
+ *   perm_gate [T*K] fp32    (out)   gate of grouped row r
+ *   slot_pos  [T, K] int32  (out)   grouped row of slot (t, k), -1 for a zero-expert slot
+ *   x_perm    [T*K, d] bf16 (out)   x_perm[r] = x[perm_tok[r]] for r < A
+ * Rows r >= A of the [T*K]-sized outputs are left untouched. */
+int moe_dispatch(const moe_dims *dims, const moe_bf16 *x, const int32_t *topk_idx,
+                 const float *topk_gate, int32_t *counts, int32_t *offsets, int32_t *perm_tok,
+                 float *perm_gate, int32_t *slot_pos, moe_bf16 *x_perm, void *ws,
+                 size_t ws_bytes, void *stream);
+
+/* The FFN experts on the grouped rows (grouped GEMMs on tcgen05 tensor cores):
+ *   h[r]      = silu(x_perm[r] W_g[e]^T) * (x_perm[r] W_u[e]^T)       bf16 [T*K, I]
+ *   y_perm[r] = perm_gate[r] * (h[r] W_d[e]^T)                          bf16 [T*K, d]
+ * for every row r in [offsets[e], offsets[e+1]) of FFN expert e (gate applied in fp32 before
+ * the bf16 rounding).  Weights in their natural layouts: W_g, W_u [N, I, d]; W_d [N, d, I].
+ * offsets must be non-decreasing with offsets[N] <= T*K (checked on the device). */
+int moe_expert_ffn(const moe_dims *dims, const moe_bf16 *x_perm, const int32_t *offsets,
+                   const float *perm_gate, const moe_bf16 *W_g, const moe_bf16 *W_u,
+                   const moe_bf16 *W_d, moe_bf16 *h, moe_bf16 *y_perm, void *ws,
+                   size_t ws_bytes, void *stream);
+
+/* Combine / un-permute: y_t = sum over FFN slots k (ascending expert id) of y_perm[slot_pos]
+ * + (sum of the zero-expert gates of t) * x_t, accumulated in fp32 in that fixed order and
+ * rounded once to bf16.  Zero experts are identities ("衝上熱搜！美團大模型，靠「快」火了",
+ * §零計算專家), so they cost one fused scalar-times-row term and no copy.
+ *   y [T, d] bf16 (out). */
+int moe_combine(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *y_perm,
+                const int32_t *topk_idx, const float *topk_gate, const int32_t *slot_pos,
+                moe_bf16 *y, void *stream);
+
+/* PID update of the FFN experts' biases from one batch's counts (same page and section, last
+ * paragraph; the law is a reading, the pages give no equation):
+ *   m = sum_{i<N} counts[i] / T;  e = (target - m) / K;  integral += e;
+ *   u = kp*e + ki*integral + kd*(e - e_prev);  e_prev = e;  b[i] += u for i < N.
+ * fp32, one rounding per operation in that order (bit-reproducible on the host).
+ *   counts    [N+Z] int32 (as written by moe_dispatch / moe_forward)
+ *   b         [N+Z] fp32  (in/out)  zero-expert biases are not changed
+ *   pid_state [2] fp32    (in/out)  {integral, e_prev}; zero-initialise before the first step
+ * T == 0 changes nothing. */
+int moe_bias_update(const moe_dims *dims, const int32_t *counts, float *b, float *pid_state,
+                    const moe_pid_params *params, void *stream);
+
+/* The whole layer in one call: moe_route, moe_dispatch, moe_expert_ffn and moe_combine on
+ * buffers carved from the workspace, with no host synchronisation.
+ *   y      [T, d] bf16 (out)
+ *   counts [N+Z] int32 (out, nullable)  per-expert slot counts of this batch, for
+ *          moe_bias_update
+ *   ws     >= moe_workspace_size(dims) bytes. */
+int moe_forward(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *W_r, const float *b,
+                const moe_bf16 *W_g, const moe_bf16 *W_u, const moe_bf16 *W_d, moe_bf16 *y,
+                int32_t *counts, void *ws, size_t ws_bytes, void *stream);
+
+/* moe_forward with timing hooks: when stage_events is not NULL it must hold
+ * MOE_NUM_STAGE_EVENTS created cudaEvent_t handles (passed as void*); event i is recorded on
+ * `stream` right before stage i is enqueued and the last one after the final stage:
+ *   0 router logits GEMM   1 softmax + biased top-K   2 dispatch (histogram, scan, permute,
+ *   gather)   3 FFN up-projection GEMM with SwiGLU   4 FFN down-projection GEMM   5 combine
+ *   6 end.
+ * Stages are enqueued exactly as by moe_forward; only the event records are added. */
+#define MOE_NUM_STAGE_EVENTS 7
+int moe_forward_timed(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *W_r,
+                      const float *b, const moe_bf16 *W_g, const moe_bf16 *W_u,
+                      const moe_bf16 *W_d, moe_bf16 *y, int32_t *counts, void *ws,
+                      size_t ws_bytes, void *const *stage_events, void *stream);
+
+/* Synchronises `stream`, returns the device status word of the workspace (MOE_DEV_* code,
+ * 0 if none) and clears it.  Returns a negative value if the synchronisation itself failed. */
+int moe_last_device_error(void *ws, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,172 @@
+// dispatch.cu -- group the FFN slots by expert: deterministic histogram, exclusive scans and a
+// stable token permutation, then a 16-byte-vectorised gather of the token rows.
+//
+// Zero-computation experts return their input ("衝上熱搜！美團大模型，靠「快」火了", §零計算專家), so
+// only slots whose expert id is < N are grouped and copied; zero-expert slots are counted (for
+// the PID controller) and get slot_pos = -1.
+//
+// Order is the stable counting sort with key (expert id, token).  Tokens are cut into chunks of
+// 256 (8 warps x 32 tokens).  In a chunk, each warp builds one 32-bit token mask per expert with
+// atomicOr (the final mask does not depend on timing), so the rank of a slot among the same
+// expert's slots is: slots in earlier chunks (column scan of the per-chunk histogram) + slots in
+// earlier warps of the chunk (popcounts) + earlier lanes of the warp (popcount of the lower mask
+// bits).  No float atomics, no spin waits: four plain kernels.
+#include "device.cuh"
+#include "kernels.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kWarps = kDispatchChunk / 32;
+
+// Masks of the chunk's tokens per (warp, expert) in shared memory: masks[w * E + e].
+__device__ __forceinline__ void build_masks(const int32_t *__restrict__ topk_idx, int T, int K,
+                                            int E, uint32_t *masks, int *status) {
+  for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) masks[i] = 0u;
+  __syncthreads();
+  const int t = blockIdx.x * kDispatchChunk + threadIdx.x;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (t < T) {
+    for (int k = 0; k < K; ++k) {
+      const int e = __ldg(topk_idx + (long long)t * K + k);
+      if (e < 0 || e >= E) {
+        record_status(status, MOE_DEV_BAD_EXPERT);
+        continue;
+      }
+      atomicOr(&masks[w * E + e], 1u << lane);
+    }
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kDispatchChunk)
+    dispatch_hist_kernel(const int32_t *__restrict__ topk_idx, int T, int K, int E,
+                         int32_t *__restrict__ chunk_counts, int *status) {
+  extern __shared__ uint32_t masks[];
+  build_masks(topk_idx, T, K, E, masks, status);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int c = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) c += __popc(masks[w * E + e]);
+    chunk_counts[(long long)blockIdx.x * E + e] = c;
+  }
+}
+
+// One block of 1024 threads (E <= 1024): column scan of the chunk histogram (in place, turning
+// counts into the chunk's starting rank per expert), expert totals, and the exclusive scan of
+// the FFN experts' totals into row offsets.
+__global__ void __launch_bounds__(1024)
+    dispatch_scan_kernel(int32_t *__restrict__ chunk_counts, int nchunks, int N, int E,
+                         int32_t *__restrict__ counts, int32_t *__restrict__ offsets) {
+  __shared__ int warp_tot[32];
+  const int e = threadIdx.x;
+  int total = 0;
+  if (e < E) {
+    for (int c = 0; c < nchunks; ++c) {
+      int32_t *p = chunk_counts + (long long)c * E + e;
+      const int v = *p;
+      *p = total;
+      total += v;
+    }
+    counts[e] = total;
+  }
+  const int v = (e < N) ? total : 0;
+  const int lane = e & 31, warp = e >> 5;
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  int base = 0;
+  for (int w = 0; w < warp; ++w) base += warp_tot[w];
+  if (e < N) offsets[e + 1] = base + incl;
+  if (e == 0) offsets[0] = 0;
+}
+
+__global__ void __launch_bounds__(kDispatchChunk)
+    dispatch_permute_kernel(const int32_t *__restrict__ topk_idx,
+                            const float *__restrict__ topk_gate, int T, int K, int N, int E,
+                            const int32_t *__restrict__ chunk_base,
+                            const int32_t *__restrict__ offsets, int32_t *__restrict__ perm_tok,
+                            float *__restrict__ perm_gate, int32_t *__restrict__ slot_pos,
+                            int *status) {
+  extern __shared__ uint32_t masks[];
+  build_masks(topk_idx, T, K, E, masks, status);
+  const int t = blockIdx.x * kDispatchChunk + threadIdx.x;
+  if (t >= T) return;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t lower = (1u << lane) - 1u;
+  for (int k = 0; k < K; ++k) {
+    const long long slot = (long long)t * K + k;
+    const int e = __ldg(topk_idx + slot);
+    if (e < 0 || e >= N) {  // zero expert (or an invalid id, already flagged)
+      slot_pos[slot] = -1;
+      continue;
+    }
+    int rank = __ldg(chunk_base + (long long)blockIdx.x * E + e);
+    for (int w2 = 0; w2 < w; ++w2) rank += __popc(masks[w2 * E + e]);
+    rank += __popc(masks[w * E + e] & lower);
+    const int r = __ldg(offsets + e) + rank;
+    perm_tok[r] = t;
+    perm_gate[r] = __ldg(topk_gate + slot);
+    slot_pos[slot] = r;
+  }
+}
+
+// x_perm[r] = x[perm_tok[r]] for r < A = offsets[N]; one warp per row, 16-byte accesses.
+__global__ void __launch_bounds__(256)
+    gather_rows_kernel(const uint4 *__restrict__ x, int d16, int T,
+                       const int32_t *__restrict__ perm_tok, const int32_t *__restrict__ a_rows,
+                       uint4 *__restrict__ x_perm, int *status) {
+  const int A = __ldg(a_rows);
+  const int warps = gridDim.x * (blockDim.x >> 5);
+  for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < A; r += warps) {
+    const int t = __ldg(perm_tok + r);
+    if (t < 0 || t >= T) {
+      if ((threadIdx.x & 31) == 0) record_status(status, MOE_DEV_BAD_ROWS);
+      continue;
+    }
+    const uint4 *src = x + (long long)t * d16;
+    uint4 *dst = x_perm + (long long)r * d16;
+    int i = threadIdx.x & 31;
+    for (; i + 96 < d16; i += 128) {
+      const uint4 v0 = __ldg(src + i), v1 = __ldg(src + i + 32), v2 = __ldg(src + i + 64),
+                  v3 = __ldg(src + i + 96);
+      dst[i] = v0;
+      dst[i + 32] = v1;
+      dst[i + 64] = v2;
+      dst[i + 96] = v3;
+    }
+    for (; i < d16; i += 32) dst[i] = __ldg(src + i);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch(const uint16_t *x, const int32_t *topk_idx, const float *topk_gate,
+                            int T, int d, int N, int E, int K, int32_t *chunk_counts,
+                            int32_t *counts, int32_t *offsets, int32_t *perm_tok,
+                            float *perm_gate, int32_t *slot_pos, uint16_t *x_perm, int *status,
+                            int num_sms, cudaStream_t stream) {
+  const int nchunks = dispatch_chunks(T);
+  const size_t mask_bytes = sizeof(uint32_t) * kWarps * E;
+  if (nchunks > 0) {
+    dispatch_hist_kernel<<<nchunks, kDispatchChunk, mask_bytes, stream>>>(topk_idx, T, K, E,
+                                                                          chunk_counts, status);
+  }
+  dispatch_scan_kernel<<<1, 1024, 0, stream>>>(chunk_counts, nchunks, N, E, counts, offsets);
+  if (nchunks > 0) {
+    dispatch_permute_kernel<<<nchunks, kDispatchChunk, mask_bytes, stream>>>(
+        topk_idx, topk_gate, T, K, N, E, chunk_counts, offsets, perm_tok, perm_gate, slot_pos,
+        status);
+    gather_rows_kernel<<<num_sms * 8, 256, 0, stream>>>(
+        reinterpret_cast<const uint4 *>(x), d / 8, T, perm_tok, offsets + N,
+        reinterpret_cast<uint4 *>(x_perm), status);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace moe

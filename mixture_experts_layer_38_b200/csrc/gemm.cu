@@ -1,0 +1,477 @@
+// gemm.cu -- persistent grouped GEMM on the sm_100a tensor cores (tcgen05.mma, TMEM
+// accumulators, TMA-fed multi-stage shared-memory ring).
+//
+// Used three ways by the MoE layer with zero-computation experts ("衝上熱搜！美團大模型，靠「快」
+// 火了", §零計算專家 and §系統級優化):
+//   router logits   l = x W_r^T                       (one group, fp32 split-K partials)
+//   FFN up          h = silu(x_perm W_g^T) * (x_perm W_u^T)    (one group per FFN expert)
+//   FFN down        y_perm = g * (h W_d^T)                     (one group per FFN expert)
+//
+// Orientation: the pages' serving stack puts the weights on the MMA's M side and the tokens on
+// N ("SwapAB"), because N may be small and irregular.  The same holds for tcgen05: with M = 128,
+// N may be any multiple of 16 up to 256, so a tile is 2 x (128 weight rows) x (n <= 128
+// tokens): two accumulators share one token tile.  For the up-projection the two weight
+// sub-tiles are 128 rows of W_g and the same 128 rows of W_u, so each TMEM lane (thread) holds
+// the gate and the up value of one feature and SwiGLU needs no data exchange.  For the down
+// projection and the router they are 256 consecutive output rows.
+//
+// Warp roles (192 threads, one CTA per SM, persistent over a static tile schedule):
+//   warp 0      TMA producer: A0/A1 weight tiles (128 x 64) and the token tile (n x 64, issued
+//               as 128/64/32/16-row boxes) into a 4-stage ring of 48 KB stages
+//   warp 1      TMEM allocator (512 columns = 2 buffers x 2 accumulators x 128) and MMA issuer
+//   warps 2-5   epilogue: tcgen05.ld from TMEM, fused SwiGLU / gate scaling / fp32 store via a
+//               per-warp shared-memory transpose and coalesced row stores
+// Tiles are ordered by group, then token tile, then weight tile, so CTAs running at the same
+// time share the token tile and walk one expert's weights together (L2 reuse).
+//
+// Every wait is bounded (device.cuh): on timeout the kernel records MOE_DEV_WAIT_TIMEOUT, all
+// roles unwind, in-flight copies and MMAs are drained (again bounded) and TMEM is freed.
+#include "device.cuh"
+#include "kernels.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kBK = 64;                      // reduction elements per stage (128-byte rows)
+constexpr int kBM = 128;                     // weight rows per MMA
+constexpr int kBN = 128;                     // max token rows per tile
+constexpr int kStages = 4;
+constexpr int kTileA = kBM * kBK * 2;        // 16 KB
+constexpr int kTileB = kBN * kBK * 2;        // 16 KB
+constexpr int kStageBytes = 2 * kTileA + kTileB;
+constexpr int kEpiWarps = 4;
+constexpr int kStagingFloats = 32 * 32;      // per epilogue warp
+constexpr int kMaxGroups = 1024;
+constexpr int kTmemCols = 512;
+constexpr long long kDrainLimitCycles = 1ll << 30;
+
+constexpr int kSmemStages = kStages * kStageBytes;
+constexpr int kSmemStaging = kEpiWarps * kStagingFloats * 4;
+constexpr int kSmemPrefix = (kMaxGroups + 4) * 4;
+constexpr int kNumBars = 2 * kStages + 4 + 1;
+constexpr int kSmemBytes = 1024 + kSmemStages + kSmemStaging + kSmemPrefix + kNumBars * 8 + 16;
+
+struct Tile {
+  int row0;     // first activation row
+  int n_valid;  // activation rows in this tile (1..128)
+  int nb;       // rows loaded / MMA N: n_valid rounded up to 16
+  int a0_row;   // first weight row of sub-tile 0 in map_a0
+  int a1_row;   // first weight row of sub-tile 1 in map_a1
+  int m0;       // first output feature of the tile
+  bool has_a1;  // sub-tile 1 exists
+  int kb0, kb1; // reduction blocks [kb0, kb1)
+  int split;
+};
+
+struct Schedule {
+  const int *prefix;  // [G + 1] token-tile prefix per group (shared memory)
+  int G;
+  int m_tiles;
+  int splits;
+  int total;
+};
+
+__device__ __forceinline__ int group_off(const GemmArgs &a, int g) {
+  if (a.group_offsets == nullptr) return g == 0 ? 0 : a.rows;
+  return __ldg(a.group_offsets + g);
+}
+
+template <int EPI>
+__device__ __forceinline__ Tile decode_tile(const GemmArgs &a, const Schedule &s, int tile) {
+  Tile t;
+  const int mt = tile % s.m_tiles;
+  const int rest = tile / s.m_tiles;
+  t.split = rest % s.splits;
+  const int ntg = rest / s.splits;
+  int lo = 0, hi = s.G - 1;  // largest g with prefix[g] <= ntg
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s.prefix[mid] <= ntg) lo = mid; else hi = mid - 1;
+  }
+  const int g = lo;
+  const int nt = ntg - s.prefix[g];
+  const int g_end = group_off(a, g + 1);
+  t.row0 = group_off(a, g) + nt * kBN;
+  t.n_valid = min(kBN, g_end - t.row0);
+  t.nb = (t.n_valid + 15) & ~15;
+  if (EPI == kEpiSwiGLU) {
+    t.m0 = mt * kBM;
+    t.a0_row = g * a.M + t.m0;
+    t.a1_row = t.a0_row;
+    t.has_a1 = true;
+  } else {
+    t.m0 = mt * 2 * kBM;
+    t.a0_row = g * a.M + t.m0;
+    t.a1_row = t.a0_row + kBM;
+    t.has_a1 = (t.m0 + kBM) < a.M;
+  }
+  const int kblocks = a.K / kBK;
+  t.kb0 = (int)(((long long)kblocks * t.split) / s.splits);
+  t.kb1 = (int)(((long long)kblocks * (t.split + 1)) / s.splits);
+  return t;
+}
+
+// Token-tile prefix over groups, computed by all threads of the block.  Returns false (and
+// records MOE_DEV_BAD_ROWS) if the offsets are not monotone or exceed the activation rows.
+__device__ bool build_schedule(const GemmArgs &a, int *prefix, int *scratch, Schedule &s) {
+  const int G = a.group_offsets ? a.num_groups : 1;
+  const int per = (G + kGemmThreads - 1) / kGemmThreads;
+  const int g_begin = min(G, (int)threadIdx.x * per);
+  const int g_end = min(G, g_begin + per);
+  int local = 0;
+  bool bad = false;
+  for (int g = g_begin; g < g_end; ++g) {
+    const int lo = group_off(a, g), hi = group_off(a, g + 1);
+    if (lo < 0 || hi < lo || hi > a.rows) { bad = true; continue; }
+    local += (hi - lo + kBN - 1) / kBN;
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = local;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) scratch[warp] = incl;
+  __syncthreads();
+  int base = 0;
+  for (int w = 0; w < warp; ++w) base += scratch[w];
+  int run = base + incl - local;
+  for (int g = g_begin; g < g_end; ++g) {
+    prefix[g] = run;
+    const int lo = group_off(a, g), hi = group_off(a, g + 1);
+    if (!(lo < 0 || hi < lo || hi > a.rows)) run += (hi - lo + kBN - 1) / kBN;
+  }
+  int total = 0;
+  for (int w = 0; w < kGemmThreads / 32; ++w) total += scratch[w];
+  if (threadIdx.x == 0) prefix[G] = total;
+  const bool any_bad = __syncthreads_or(bad);
+  if (any_bad && threadIdx.x == 0) record_status(a.status, MOE_DEV_BAD_ROWS);
+  s.prefix = prefix;
+  s.G = G;
+  s.total = any_bad ? 0 : total;
+  return !any_bad;
+}
+
+template <int EPI>
+__device__ __forceinline__ int m_tiles_of(int M) {
+  return EPI == kEpiSwiGLU ? (M + kBM - 1) / kBM : (M + 2 * kBM - 1) / (2 * kBM);
+}
+
+// Bounded wait by lane 0 of a warp, result broadcast so the warp stays converged.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+  int ok = 0;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+__device__ __forceinline__ void signal_abort(const GemmArgs &a, volatile int *abort) {
+  record_status(a.status, MOE_DEV_WAIT_TIMEOUT);
+  *abort = 1;
+}
+
+__device__ __forceinline__ float silu(float z) { return z / (1.0f + __expf(-z)); }
+
+// ------------------------------------------------------------------ epilogue, one 32-token chunk
+// Thread `lane` of epilogue warp with TMEM lane quarter q owns output feature (q*32 + lane) of
+// each 128-row sub-tile; after the transpose through `stage` each thread stores 16 bytes of a
+// token row.
+template <int EPI>
+__device__ __forceinline__ void epilogue_chunk(const GemmArgs &a, const Tile &t, uint32_t tcol,
+                                               int chunk, int q, int lane, float *stage) {
+  const int tok0 = chunk * 32;
+  if (EPI == kEpiSwiGLU) {
+    uint32_t g[32], u[32];
+    tmem_ld_32x32b_x32(tcol, g);
+    tmem_ld_32x32b_x32(tcol + kBM, u);
+    tmem_ld_wait();
+    uint16_t *st = reinterpret_cast<uint16_t *>(stage);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float h = silu(__uint_as_float(g[j])) * __uint_as_float(u[j]);
+      st[j * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(h));
+    }
+    __syncwarp();
+    const int f = t.m0 + q * 32 + (lane & 3) * 8;
+    uint16_t *out = reinterpret_cast<uint16_t *>(a.out);
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+      const int r = it * 8 + (lane >> 2);
+      const int tok = tok0 + r;
+      if (tok < t.n_valid && f < a.M) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(st + r * 32 + (lane & 3) * 8);
+        *reinterpret_cast<uint4 *>(out + (long long)(t.row0 + tok) * a.out_ld + f) = v;
+      }
+    }
+    __syncwarp();
+  } else {
+    float gate = 0.f;
+    if (EPI == kEpiGated) {
+      const int tok = tok0 + lane;
+      gate = tok < t.n_valid ? __ldg(a.row_scale + t.row0 + tok) : 0.f;
+    }
+#pragma unroll 1
+    for (int sub = 0; sub < 2; ++sub) {
+      if (sub == 1 && !t.has_a1) break;
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tcol + sub * kBM, v);
+      tmem_ld_wait();
+      const int fbase = t.m0 + sub * kBM + q * 32;
+      if (EPI == kEpiGated) {
+        uint16_t *st = reinterpret_cast<uint16_t *>(stage);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float gj = __shfl_sync(0xffffffffu, gate, j);
+          st[j * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j]) * gj));
+        }
+        __syncwarp();
+        const int f = fbase + (lane & 3) * 8;
+        uint16_t *out = reinterpret_cast<uint16_t *>(a.out);
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+          const int r = it * 8 + (lane >> 2);
+          const int tok = tok0 + r;
+          if (tok < t.n_valid && f < a.M) {
+            const uint4 val = *reinterpret_cast<const uint4 *>(st + r * 32 + (lane & 3) * 8);
+            *reinterpret_cast<uint4 *>(out + (long long)(t.row0 + tok) * a.out_ld + f) = val;
+          }
+        }
+        __syncwarp();
+      } else {  // kEpiF32
+#pragma unroll
+        for (int j = 0; j < 32; ++j) stage[j * 32 + lane] = __uint_as_float(v[j]);
+        __syncwarp();
+        const int f = fbase + (lane & 7) * 4;
+        float *out = reinterpret_cast<float *>(a.out) + (long long)t.split * a.split_stride;
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+          const int r = it * 4 + (lane >> 3);
+          const int tok = tok0 + r;
+          if (tok < t.n_valid && f < a.M) {
+            const float4 val = *reinterpret_cast<const float4 *>(stage + r * 32 + (lane & 7) * 4);
+            *reinterpret_cast<float4 *>(out + (long long)(t.row0 + tok) * a.out_ld + f) = val;
+          }
+        }
+        __syncwarp();
+      }
+    }
+  }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ GemmArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *ring = smem;
+  float *staging = reinterpret_cast<float *>(smem + kSmemStages);
+  int *prefix = reinterpret_cast<int *>(smem + kSmemStages + kSmemStaging);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kSmemStages + kSmemStaging + kSmemPrefix);
+  uint64_t *full_bar = bars;
+  uint64_t *empty_bar = bars + kStages;
+  uint64_t *tfull_bar = bars + 2 * kStages;
+  uint64_t *tempty_bar = bars + 2 * kStages + 2;
+  uint64_t *drain_bar = bars + 2 * kStages + 4;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kNumBars);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull_bar[b], 1);
+      mbar_init(&tempty_bar[b], kEpiWarps);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&args.map_a0);
+    tma_prefetch_desc(&args.map_a1);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) tma_prefetch_desc(&args.map_b[i]);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  Schedule sched;
+  build_schedule(args, prefix, reinterpret_cast<int *>(staging), sched);
+  sched.m_tiles = m_tiles_of<EPI>(args.M);
+  sched.splits = EPI == kEpiF32 ? args.k_splits : 1;
+  sched.total = sched.total * sched.m_tiles * sched.splits;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      const uint64_t pol_w = l2_policy_evict_normal();
+      const uint64_t pol_x = l2_policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      long long issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < sched.total; tile += gridDim.x) {
+        const Tile t = decode_tile<EPI>(args, sched, tile);
+        const uint32_t bytes = kTileA * (t.has_a1 ? 2 : 1) + t.nb * kBK * 2;
+        for (int kb = t.kb0; kb < t.kb1; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag)) {
+            signal_abort(args, abort_flag);
+            ok = false;
+            break;
+          }
+          uint8_t *sa0 = ring + stage * kStageBytes;
+          uint8_t *sa1 = sa0 + kTileA;
+          uint8_t *sb = sa0 + 2 * kTileA;
+          const int kc = kb * kBK;
+          mbar_arrive_expect_tx(&full_bar[stage], bytes);
+          tma_load_2d(sa0, &args.map_a0, &full_bar[stage], kc, t.a0_row, pol_w);
+          if (t.has_a1) tma_load_2d(sa1, &args.map_a1, &full_bar[stage], kc, t.a1_row, pol_w);
+          int r = 0;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int box = kBN >> i;
+            if (t.nb - r >= box) {
+              tma_load_2d(sb + r * (kBK * 2), &args.map_b[i], &full_bar[stage], kc, t.row0 + r,
+                          pol_x);
+              r += box;
+            }
+          }
+          ++issued;
+          if (++stage == kStages) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (!ok) {
+        // Drain the copies that may still be landing in the ring (bounded).
+        for (long long i = 1; i <= issued && i <= kStages; ++i) {
+          const long long idx = issued - i;
+          const int s = (int)(idx % kStages);
+          const uint32_t par = (uint32_t)((idx / kStages) & 1);
+          const long long t0 = clock64();
+          while (!mbar_try_wait(&full_bar[s], par) && clock64() - t0 < kDrainLimitCycles) {}
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      bool any = false;
+      for (int tile = blockIdx.x; ok && tile < sched.total; tile += gridDim.x, ++it) {
+        const Tile t = decode_tile<EPI>(args, sched, tile);
+        const int buf = it & 1;
+        const uint32_t use = (uint32_t)(it >> 1);
+        if (!mbar_wait(&tempty_bar[buf], (use & 1) ^ 1, abort_flag)) {
+          signal_abort(args, abort_flag);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + buf * (2 * kBM);
+        const uint32_t d1 = d0 + kBM;
+        const uint32_t idesc = idesc_bf16_f32(kBM, t.nb);
+        for (int kb = t.kb0; kb < t.kb1; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, abort_flag)) {
+            signal_abort(args, abort_flag);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t base = smem_u32(ring + stage * kStageBytes);
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            const uint64_t bdesc = sw128_kmajor_desc(base + 2 * kTileA + k * 32);
+            const uint32_t acc = (kb > t.kb0 || k > 0) ? 1u : 0u;
+            umma_bf16(d0, sw128_kmajor_desc(base + k * 32), bdesc, idesc, acc);
+            if (t.has_a1) umma_bf16(d1, sw128_kmajor_desc(base + kTileA + k * 32), bdesc, idesc, acc);
+          }
+          any = true;
+          umma_commit(&empty_bar[stage]);
+          if (++stage == kStages) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        umma_commit(&tfull_bar[buf]);
+      }
+      if (!ok && any) {
+        umma_commit(drain_bar);
+        const long long t0 = clock64();
+        while (!mbar_try_wait(drain_bar, 0) && clock64() - t0 < kDrainLimitCycles) {}
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue warps
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    float *stage = staging + (warp - 2) * kStagingFloats;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < sched.total; tile += gridDim.x, ++it) {
+      const Tile t = decode_tile<EPI>(args, sched, tile);
+      const int buf = it & 1;
+      const uint32_t use = (uint32_t)(it >> 1);
+      if (!warp_wait(&tfull_bar[buf], use & 1, abort_flag)) {
+        if (lane == 0) signal_abort(args, abort_flag);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tcol = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * (2 * kBM);
+      const int chunks = (t.n_valid + 31) / 32;
+      for (int c = 0; c < chunks; ++c) epilogue_chunk<EPI>(args, t, tcol + c * 32, c, q, lane, stage);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty_bar[buf]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace
+
+int gemm_smem_bytes() { return kSmemBytes; }
+
+cudaError_t gemm_prepare(int device) {
+  (void)device;
+  cudaError_t e;
+  e = cudaFuncSetAttribute(grouped_gemm_kernel<kEpiSwiGLU>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(grouped_gemm_kernel<kEpiGated>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(grouped_gemm_kernel<kEpiF32>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+}
+
+cudaError_t launch_grouped_gemm(int epi, const GemmArgs &args, int grid, cudaStream_t stream) {
+  switch (epi) {
+    case kEpiSwiGLU:
+      grouped_gemm_kernel<kEpiSwiGLU><<<grid, kGemmThreads, kSmemBytes, stream>>>(args);
+      break;
+    case kEpiGated:
+      grouped_gemm_kernel<kEpiGated><<<grid, kGemmThreads, kSmemBytes, stream>>>(args);
+      break;
+    default:
+      grouped_gemm_kernel<kEpiF32><<<grid, kGemmThreads, kSmemBytes, stream>>>(args);
+      break;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,63 @@
+// kernels.cuh -- host-side launchers of the library's kernels (internal C++ interface between
+// the C ABI in moe_api.cu and the kernel files).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+// ------------------------------------------------------------------ grouped GEMM (tcgen05)
+// Output tile = 2 x (128 weight rows) x (<= 128 activation rows); see gemm.cu.
+enum EpiKind : int {
+  kEpiSwiGLU = 0,  // h = silu(A0 x) * (A1 x)           -> bf16 [rows, M]
+  kEpiGated = 1,   // y = row_scale[r] * (A x)          -> bf16 [rows, M]
+  kEpiF32 = 2      // logits (split-K partials)         -> fp32 [splits][rows, M]
+};
+
+struct GemmArgs {
+  CUtensorMap map_a0;    // weight rows (box 64 x 128)
+  CUtensorMap map_a1;    // W_u for SwiGLU, the same tensor as map_a0 otherwise
+  CUtensorMap map_b[4];  // activation rows, boxes of 128 / 64 / 32 / 16 rows x 64 columns
+  const int32_t *group_offsets;  // [num_groups + 1] activation-row offsets, or nullptr
+  int num_groups;                // groups (experts); 1 when group_offsets == nullptr
+  int rows;                      // activation rows available (bound for group_offsets)
+  int M;                         // weight rows per group that produce outputs
+  int K;                         // reduction length, a multiple of 64
+  int k_splits;                  // split-K factor (kEpiF32 only)
+  void *out;
+  int out_ld;                    // elements per output row
+  long long split_stride;        // elements between split-K partial outputs
+  const float *row_scale;        // kEpiGated: per-row gate
+  int *status;                   // device status word
+};
+
+constexpr int kGemmThreads = 192;
+int gemm_smem_bytes();
+cudaError_t gemm_prepare(int device);  // sets the kernels' shared-memory limit once per device
+cudaError_t launch_grouped_gemm(int epi, const GemmArgs &args, int grid, cudaStream_t stream);
+
+// ------------------------------------------------------------------ routing
+// logits [splits][T][E] fp32 -> softmax, biased top-K, ascending ids.
+cudaError_t launch_route_topk(const float *logits, int splits, int T, int E, int K,
+                              const float *b, int32_t *topk_idx, float *topk_gate, float *gap,
+                              int *status, cudaStream_t stream);
+
+// ------------------------------------------------------------------ dispatch
+constexpr int kDispatchChunk = 256;  // tokens per histogram chunk (8 warps x 32)
+inline int dispatch_chunks(int T) { return (T + kDispatchChunk - 1) / kDispatchChunk; }
+cudaError_t launch_dispatch(const uint16_t *x, const int32_t *topk_idx, const float *topk_gate,
+                            int T, int d, int N, int E, int K, int32_t *chunk_counts,
+                            int32_t *counts, int32_t *offsets, int32_t *perm_tok,
+                            float *perm_gate, int32_t *slot_pos, uint16_t *x_perm, int *status,
+                            int num_sms, cudaStream_t stream);
+
+// ------------------------------------------------------------------ combine and PID
+cudaError_t launch_combine(const uint16_t *x, const uint16_t *y_perm, const int32_t *topk_idx,
+                           const float *topk_gate, const int32_t *slot_pos, int T, int d, int N,
+                           int K, int rows, uint16_t *y, int *status, cudaStream_t stream);
+cudaError_t launch_pid(const int32_t *counts, int N, int K, int T, float *b, float *state,
+                       float target, float kp, float ki, float kd, cudaStream_t stream);
+
+}  // namespace moe

@@ -89,6 +89,14 @@ def _normal_bf16(gen, shape, std, dev):
         torch.bfloat16)
 
 
+def apply_zipf_router(w: Workload, W_r: torch.Tensor) -> torch.Tensor:
+    """In place: column 0 of W_r becomes -s * ln(i + 1), the Zipf(s) logit offset of expert i
+    (tokens of a Zipf workload carry a constant 1 in feature 0)."""
+    ranks = torch.arange(1, W_r.shape[0] + 1, dtype=torch.float64, device=W_r.device)
+    W_r[:, 0] = (-w.zipf_s * torch.log(ranks)).to(torch.bfloat16)
+    return W_r
+
+
 def make_weights(w: Workload, device="cpu", seed: int = 0) -> dict:
     """W_r [E,d], b [E] fp32, W_g/W_u [N,I,d], W_d [N,d,I] (bf16), all on ``device``."""
     gdev = _gen_device(w, device)
@@ -101,8 +109,7 @@ def make_weights(w: Workload, device="cpu", seed: int = 0) -> dict:
     else:
         b = torch.zeros((w.E,), dtype=torch.float32, device=gdev)
     if w.zipf_s > 0:
-        ranks = torch.arange(1, w.E + 1, dtype=torch.float64, device=gdev)
-        W_r[:, 0] = (-w.zipf_s * torch.log(ranks)).to(torch.bfloat16)
+        apply_zipf_router(w, W_r)
     W_g = torch.empty((w.N, w.I, w.d), dtype=torch.bfloat16, device=device)
     W_u = torch.empty((w.N, w.I, w.d), dtype=torch.bfloat16, device=device)
     W_d = torch.empty((w.N, w.d, w.I), dtype=torch.bfloat16, device=device)

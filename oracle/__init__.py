@@ -38,10 +38,13 @@ def _load():
                                                _ptr, _ptr, _ptr, _ptr, _ptr]
         _lib.oracle_forward.argtypes = [_i64, _i64, _i64, _i64, _i64, _i64, _ptr, _ptr, _ptr,
                                         _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _ptr]
+        _lib.oracle_combine_rows.argtypes = [_i64, _i64, _i64, _i64, _ptr, _ptr, _ptr, _ptr,
+                                             _ptr, _ptr]
         _lib.oracle_pid_step.argtypes = [_i64, _i64, _i64, _ptr, _ptr, _ptr, ctypes.c_float,
                                          ctypes.c_float, ctypes.c_float, ctypes.c_float]
         for f in ("oracle_router", "oracle_dispatch", "oracle_swiglu_expert",
-                  "oracle_combine_tokens", "oracle_forward", "oracle_pid_step"):
+                  "oracle_combine_tokens", "oracle_combine_rows", "oracle_forward",
+                  "oracle_pid_step"):
             getattr(_lib, f).restype = None
     return _lib
 
@@ -143,6 +146,23 @@ def combine_tokens(tokens, x, topk_idx, topk_gate, W_g, W_u, W_d, N):
     y = np.zeros((len(tokens), d), np.float64)
     _load().oracle_combine_tokens(d, N, K, I, len(tokens), _p(tokens), _p(x), _p(topk_idx),
                                   _p(topk_gate), _p(W_g), _p(W_u), _p(W_d), _p(y))
+    return y
+
+
+def combine_rows(x, topk_idx, topk_gate, slot_pos, rows, N):
+    """y_t = sum_k (FFN slot: rows[slot_pos[t,k]], zero slot: g_{t,k} x_t); rows are already gated."""
+    x = bf16_bits(x)
+    topk_idx, slot_pos = _i32(topk_idx), _i32(slot_pos)
+    topk_gate = np.ascontiguousarray(topk_gate, dtype=np.float64)
+    rows = np.ascontiguousarray(rows, dtype=np.float64)
+    T, d = x.shape
+    K = topk_idx.shape[1]
+    assert rows.ndim == 2 and rows.shape[1] == d
+    ffn = topk_idx < N
+    assert (slot_pos[ffn] >= 0).all() and (slot_pos[ffn] < max(len(rows), 1)).all()
+    y = np.zeros((T, d), np.float64)
+    _load().oracle_combine_rows(T, d, N, K, _p(x), _p(topk_idx), _p(topk_gate), _p(slot_pos),
+                                _p(rows), _p(y))
     return y
 
 

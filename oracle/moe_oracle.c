@@ -240,6 +240,33 @@ void oracle_combine_tokens(int64_t d, int64_t N, int64_t K, int64_t I, int64_t n
     }
 }
 
+/* ------------------------------------------------------------------------------------------
+ * The weighted sum alone, for given expert outputs (P1 §零計算專家):
+ *   y_t = sum_{k < K} ( i_{t,k} < N ? rows[slot_pos[t,k]] : g_{t,k} * x_t )
+ * where rows[r] already holds g * E_i(x) for grouped row r (the FFN terms arrive gated), and
+ * slot_pos maps slot (t, k) to its grouped row.  Slots summed in order, fp64.
+ * ---------------------------------------------------------------------------------------- */
+void oracle_combine_rows(int64_t T, int64_t d, int64_t N, int64_t K, const uint16_t *x,
+                         const int32_t *topk_idx, const double *topk_gate,
+                         const int32_t *slot_pos, const double *rows, double *y)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        double *yt = y + t * d;
+        for (int64_t j = 0; j < d; ++j) yt[j] = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            int32_t i = topk_idx[t * K + k];
+            if (i >= N) {
+                double g = topk_gate[t * K + k];
+                for (int64_t j = 0; j < d; ++j) yt[j] += g * bf16_to_f64(x[t * d + j]);
+            } else {
+                const double *r = rows + (int64_t)slot_pos[t * K + k] * d;
+                for (int64_t j = 0; j < d; ++j) yt[j] += r[j];
+            }
+        }
+    }
+}
+
 /* Router, then the layer, for all T tokens. */
 void oracle_forward(int64_t T, int64_t d, int64_t N, int64_t Z, int64_t K, int64_t I,
                     const uint16_t *x, const uint16_t *W_r, const float *b, const uint16_t *W_g,

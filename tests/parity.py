@@ -1,0 +1,136 @@
+"""Shared helpers for the GPU parity tests: run the CUDA path through the C ABI and compare it
+with the CPU oracle under the layer's parity rules.
+
+Parity rules (from the layer's specification):
+  * routing: for every token whose oracle gap s_(K) - s_(K+1) exceeds 1e-4 the selected ids
+    are bit-exact; tokens at or below it are near-ties, counted, and the GPU's set must be
+    eps-valid: min over selected oracle scores >= max over unselected oracle scores - 1e-4;
+  * dispatch (counts, offsets, permutation, slot rows): bit-exact;
+  * outputs: max|y - y_ref| <= 1e-2 * max|y_ref| and ||y - y_ref||_2 <= 5e-3 * ||y_ref||_2.
+Gate values come from an fp32 softmax on the GPU and an fp64 one in the oracle; they are
+compared with a relative tolerance of 2e-5 (fp32 logits of a d-term dot product, then exp).
+"""
+import numpy as np
+import torch
+
+import oracle
+from mixture_experts_layer_38_b200 import binding as mb
+
+GAP_EPS = 1e-4
+Y_MAX_TOL = 1e-2
+Y_L2_TOL = 5e-3
+GATE_RTOL = 2e-5
+
+
+def y_errors(y, y_ref):
+    y = np.asarray(y, np.float64)
+    y_ref = np.asarray(y_ref, np.float64)
+    max_ref = np.abs(y_ref).max()
+    max_err = np.abs(y - y_ref).max()
+    l2 = np.linalg.norm(y - y_ref) / max(np.linalg.norm(y_ref), 1e-300)
+    return max_err / max(max_ref, 1e-300), l2
+
+
+def assert_y_close(y, y_ref, what="y"):
+    rel_max, rel_l2 = y_errors(y, y_ref)
+    assert rel_max <= Y_MAX_TOL and rel_l2 <= Y_L2_TOL, (
+        f"{what}: max|err|/max|ref| = {rel_max:.3e} (<= {Y_MAX_TOL}), "
+        f"relative L2 = {rel_l2:.3e} (<= {Y_L2_TOL})")
+    return rel_max, rel_l2
+
+
+def check_routing(gpu_idx, gpu_gate, ref, scores=None):
+    """Compare GPU top-K with the oracle's.  Returns (near_tie_count, mismatched_near_ties).
+
+    ``ref`` is oracle.router output for the same rows; ``scores`` the oracle's full biased
+    scores (needed only to validate near-tie tokens whose GPU set differs)."""
+    gpu_idx = np.asarray(gpu_idx)
+    gpu_gate = np.asarray(gpu_gate, np.float64)
+    clear = ref["gap"] > GAP_EPS
+    np.testing.assert_array_equal(gpu_idx[clear], ref["topk_idx"][clear])
+    same = (gpu_idx == ref["topk_idx"]).all(axis=1)
+    np.testing.assert_allclose(gpu_gate[same], ref["topk_gate"][same], rtol=GATE_RTOL, atol=1e-30)
+    differ = np.flatnonzero(~same)
+    for t in differ:
+        assert scores is not None, "near-tie token selected differently; scores needed"
+        s = scores[t]
+        sel = np.zeros(len(s), bool)
+        sel[gpu_idx[t]] = True
+        assert len(set(gpu_idx[t].tolist())) == gpu_idx.shape[1]
+        assert (np.diff(gpu_idx[t]) > 0).all()
+        assert s[sel].min() >= s[~sel].max() - GAP_EPS, f"token {t}: GPU set is not eps-valid"
+    return int((~clear).sum()), len(differ)
+
+
+def check_dispatch_properties(idx, counts, offsets, perm_tok, slot_pos, N, E):
+    """The GPU dispatch must be exactly the stable (expert, token) sort of its own routing."""
+    idx = np.asarray(idx)
+    T, K = idx.shape
+    np.testing.assert_array_equal(counts, np.bincount(idx.reshape(-1), minlength=E))
+    ex = idx.reshape(-1)
+    tok = np.repeat(np.arange(T), K)
+    ffn = ex < N
+    order = np.lexsort((tok[ffn], ex[ffn]))
+    A = int(ffn.sum())
+    np.testing.assert_array_equal(offsets, np.concatenate([[0], np.cumsum(counts[:N])]))
+    np.testing.assert_array_equal(perm_tok[:A], tok[ffn][order])
+    rows = np.full(T * K, -1)
+    rows[np.flatnonzero(ffn)[order]] = np.arange(A)
+    np.testing.assert_array_equal(np.asarray(slot_pos).reshape(-1), rows)
+
+
+def to_np(t):
+    if t.dtype == torch.bfloat16:
+        return oracle.bf16_bits(t)
+    return t.detach().cpu().numpy()
+
+
+class Stages:
+    """Device buffers for running the staged C-ABI calls on one workload."""
+
+    def __init__(self, w, x, wt, device="cuda"):
+        self.w = w
+        self.dm = mb.dims(w.T, w.d, w.N, w.Z, w.K, w.I)
+        R = w.T * w.K
+        i32 = dict(dtype=torch.int32, device=device)
+        f32 = dict(dtype=torch.float32, device=device)
+        bf = dict(dtype=torch.bfloat16, device=device)
+        self.x = x.to(device)
+        self.wt = {k: v.to(device) for k, v in wt.items()}
+        self.ws = mb.alloc_workspace(self.dm, device)
+        self.topk_idx = torch.zeros((w.T, w.K), **i32)
+        self.topk_gate = torch.zeros((w.T, w.K), **f32)
+        self.gap = torch.zeros((w.T,), **f32)
+        self.counts = torch.zeros((w.E,), **i32)
+        self.offsets = torch.zeros((w.N + 1,), **i32)
+        self.perm_tok = torch.full((R,), -7, **i32)
+        self.perm_gate = torch.zeros((R,), **f32)
+        self.slot_pos = torch.zeros((w.T, w.K), **i32)
+        self.x_perm = torch.zeros((R, w.d), **bf)
+        self.h = torch.zeros((R, w.I), **bf)
+        self.y_perm = torch.zeros((R, w.d), **bf)
+        self.y = torch.zeros((w.T, w.d), **bf)
+
+    def route(self, b=None):
+        mb.moe_route(self.dm, self.x, self.wt["W_r"], self.wt["b"] if b is None else b,
+                     self.topk_idx, self.topk_gate, self.gap, self.ws)
+
+    def dispatch(self):
+        mb.moe_dispatch(self.dm, self.x, self.topk_idx, self.topk_gate, self.counts, self.offsets,
+                        self.perm_tok, self.perm_gate, self.slot_pos, self.x_perm, self.ws)
+
+    def expert_ffn(self):
+        mb.moe_expert_ffn(self.dm, self.x_perm, self.offsets, self.perm_gate, self.wt["W_g"],
+                          self.wt["W_u"], self.wt["W_d"], self.h, self.y_perm, self.ws)
+
+    def combine(self):
+        mb.moe_combine(self.dm, self.x, self.y_perm, self.topk_idx, self.topk_gate,
+                       self.slot_pos, self.y)
+
+    def forward(self, b=None, counts=None):
+        mb.moe_forward(self.dm, self.x, self.wt["W_r"], self.wt["b"] if b is None else b,
+                       self.wt["W_g"], self.wt["W_u"], self.wt["W_d"], self.y,
+                       self.counts if counts is None else counts, self.ws)
+
+    def device_status(self):
+        return mb.moe_last_device_error(self.ws)

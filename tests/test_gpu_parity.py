@@ -1,0 +1,300 @@
+"""GPU parity: every stage of the CUDA path, called through the C ABI, against the CPU oracle.
+
+Stage tests feed the GPU stage the oracle's own upstream results (never the other way round),
+so each kernel is checked in isolation; end-to-end tests compare moe_forward with the oracle
+on the same seeded inputs.  Workloads: tiny (whole batch), mid (sampled tokens), and edge
+cases (T = 0, ragged T, one token, all-zero-expert routing, one expert holding every token,
+K = N + Z, widths that are not multiples of the 128-row tiles).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mixture_experts_layer_38_b200 import binding as mb
+from mixture_experts_layer_38_b200.workloads import WORKLOADS, Workload, make_tokens, make_weights
+from parity import (Stages, assert_y_close, check_dispatch_properties, check_routing, to_np)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _case(w, seed=0, bias=None, T=None):
+    wt = make_weights(w, seed=seed)
+    if bias is not None:
+        wt["b"] = bias
+    x = make_tokens(w, seed=seed, T=T)
+    if T is not None:
+        w = Workload(w.name, T=T, d=w.d, N=w.N, Z=w.Z, K=w.K, I=w.I, bias_range=w.bias_range)
+    return w, x, wt
+
+
+def _oracle_expert_rows(w, x, wt, ref_idx, ref_gate, dsp):
+    """g_r * E_e(x_t) per grouped row, from the oracle (fp64)."""
+    xb = oracle.bf16_bits(x)
+    A = len(dsp["perm_tok"])
+    gates = np.zeros(A)
+    T, K = ref_idx.shape
+    for t in range(T):
+        for k in range(K):
+            r = dsp["slot_pos"][t, k]
+            if r >= 0:
+                gates[r] = np.float32(ref_gate[t, k])  # the fp32 gate the GPU stage is given
+    rows = np.zeros((A, w.d))
+    for e in range(w.N):
+        lo, hi = dsp["offsets"][e], dsp["offsets"][e + 1]
+        if hi > lo:
+            out = oracle.swiglu_expert(xb[dsp["perm_tok"][lo:hi]], wt["W_g"][e], wt["W_u"][e],
+                                       wt["W_d"][e])
+            rows[lo:hi] = gates[lo:hi, None] * out
+    return rows, gates
+
+
+# ---------------------------------------------------------------------------------- stages
+@pytest.mark.parametrize("name", ["tiny", "mid"])
+def test_route_matches_oracle(name):
+    w = WORKLOADS[name]
+    w, x, wt = _case(w, T=512 if name == "mid" else None)
+    st = Stages(w, x, wt)
+    st.route()
+    ref = oracle.router(x, wt["W_r"], wt["b"], w.K, want_scores=True)
+    near, differ = check_routing(to_np(st.topk_idx), to_np(st.topk_gate), ref, ref["scores"])
+    gap = to_np(st.gap).astype(np.float64)
+    np.testing.assert_allclose(gap, ref["gap"], rtol=0, atol=2e-6)
+    assert st.device_status() == 0
+    print(f"{name}: near-ties {near}/{w.T}, differing near-ties {differ}")
+
+
+@pytest.mark.parametrize("name", ["tiny", "mid"])
+def test_dispatch_matches_oracle(name):
+    w = WORKLOADS[name]
+    w, x, wt = _case(w, T=1000 if name == "mid" else None)
+    ref = oracle.router(x, wt["W_r"], wt["b"], w.K)
+    dsp = oracle.dispatch(ref["topk_idx"], w.N, w.E)
+    st = Stages(w, x, wt)
+    st.topk_idx.copy_(torch.from_numpy(ref["topk_idx"]))
+    st.topk_gate.copy_(torch.from_numpy(ref["topk_gate"].astype(np.float32)))
+    st.dispatch()
+    A = len(dsp["perm_tok"])
+    np.testing.assert_array_equal(to_np(st.counts), dsp["counts"])
+    np.testing.assert_array_equal(to_np(st.offsets), dsp["offsets"])
+    np.testing.assert_array_equal(to_np(st.perm_tok)[:A], dsp["perm_tok"])
+    np.testing.assert_array_equal(to_np(st.slot_pos), dsp["slot_pos"])
+    assert (to_np(st.perm_tok)[A:] == -7).all()  # rows past A untouched
+    g32 = ref["topk_gate"].astype(np.float32)
+    want_gate = np.zeros(A, np.float32)
+    ffn = dsp["slot_pos"] >= 0
+    want_gate[dsp["slot_pos"][ffn]] = g32[ffn]
+    np.testing.assert_array_equal(to_np(st.perm_gate)[:A], want_gate)
+    np.testing.assert_array_equal(to_np(st.x_perm)[:A], oracle.bf16_bits(x)[dsp["perm_tok"]])
+    assert st.device_status() == 0
+
+
+@pytest.mark.parametrize("name", ["tiny", "mid"])
+def test_expert_ffn_matches_oracle(name):
+    w = WORKLOADS[name]
+    w, x, wt = _case(w, T=256 if name == "mid" else None)
+    ref = oracle.router(x, wt["W_r"], wt["b"], w.K)
+    dsp = oracle.dispatch(ref["topk_idx"], w.N, w.E)
+    rows, gates = _oracle_expert_rows(w, x, wt, ref["topk_idx"], ref["topk_gate"], dsp)
+    A = len(dsp["perm_tok"])
+    st = Stages(w, x, wt)
+    st.x_perm[:A].copy_(x[torch.from_numpy(dsp["perm_tok"]).long()])
+    st.offsets.copy_(torch.from_numpy(dsp["offsets"]))
+    st.perm_gate[:A].copy_(torch.from_numpy(gates.astype(np.float32)))
+    st.expert_ffn()
+    got = to_np(st.y_perm)[:A]
+    assert_y_close(oracle.bf16_to_f64(got), rows, f"{name} y_perm")
+    assert st.device_status() == 0
+
+
+@pytest.mark.parametrize("name", ["tiny", "mid"])
+def test_combine_matches_oracle(name):
+    w = WORKLOADS[name]
+    w, x, wt = _case(w, T=300 if name == "mid" else None)
+    ref = oracle.router(x, wt["W_r"], wt["b"], w.K)
+    dsp = oracle.dispatch(ref["topk_idx"], w.N, w.E)
+    A = len(dsp["perm_tok"])
+    # Arbitrary seeded expert-output rows (combine does not care where they come from).
+    g = torch.Generator().manual_seed(11)
+    y_perm = torch.randn((w.T * w.K, w.d), generator=g).to(torch.bfloat16)
+    st = Stages(w, x, wt)
+    st.y_perm.copy_(y_perm)
+    st.topk_idx.copy_(torch.from_numpy(ref["topk_idx"]))
+    st.topk_gate.copy_(torch.from_numpy(ref["topk_gate"].astype(np.float32)))
+    st.slot_pos.copy_(torch.from_numpy(dsp["slot_pos"]))
+    st.combine()
+    rows = oracle.bf16_to_f64(oracle.bf16_bits(y_perm))[:max(A, 1)]
+    want = oracle.combine_rows(x, ref["topk_idx"], ref["topk_gate"].astype(np.float32),
+                               dsp["slot_pos"], rows, w.N)
+    got = oracle.bf16_to_f64(to_np(st.y))
+    assert_y_close(got, want, f"{name} combine")
+    # fp32 accumulation then one bf16 rounding: within 2^-8 relative of each element (+ abs eps)
+    assert (np.abs(got - want) <= 2.0 ** -8 * np.abs(want) + 1e-3 * np.abs(want).max()).all()
+
+
+def test_pid_matches_oracle_bit_exact():
+    w = WORKLOADS["skewed"]
+    dm = mb.dims(w.T, w.d, w.N, w.Z, w.K, w.I)
+    rng = np.random.default_rng(5)
+    b = (rng.uniform(-0.05, 0.05, w.E)).astype(np.float32)
+    st = np.zeros(2, np.float32)
+    b_gpu = torch.from_numpy(b.copy()).to(DEV)
+    st_gpu = torch.zeros(2, dtype=torch.float32, device=DEV)
+    params = mb.PidParams(8.0, 0.005, 0.002, 0.001)
+    for step in range(20):
+        counts = rng.integers(0, 400, w.E).astype(np.int32)
+        mb.moe_bias_update(dm, torch.from_numpy(counts).to(DEV), b_gpu, st_gpu, params)
+        oracle.pid_step(counts, b, st, w.N, w.K, w.T, 8.0, 0.005, 0.002, 0.001)
+        assert b_gpu.cpu().numpy().tobytes() == b.tobytes(), step
+        assert st_gpu.cpu().numpy().tobytes() == st.tobytes(), step
+
+
+# ---------------------------------------------------------------------------------- end to end
+def _forward_vs_oracle(w, x, wt, sample=None, seed=0):
+    st = Stages(w, x, wt)
+    st.forward()
+    y = oracle.bf16_to_f64(to_np(st.y))
+    counts = to_np(st.counts)
+    assert counts.sum() == w.T * w.K
+    tokens = np.arange(w.T) if sample is None else np.sort(
+        np.random.default_rng(seed).choice(w.T, sample, replace=False))
+    ref = oracle.forward_sampled(tokens, x, wt["W_r"], wt["b"], w.N, w.Z, w.K,
+                                 lambda e: (wt["W_g"][e], wt["W_u"][e], wt["W_d"][e]))
+    # Routing of the sampled tokens, from the staged route call (same kernels as moe_forward).
+    st.route()
+    idx = to_np(st.topk_idx)[tokens]
+    scores = oracle.router(oracle.bf16_bits(x)[tokens], wt["W_r"], wt["b"], w.K,
+                           want_scores=True)["scores"]
+    near, differ = check_routing(idx, to_np(st.topk_gate)[tokens], ref, scores)
+    same = (idx == ref["topk_idx"]).all(axis=1)
+    assert_y_close(y[tokens][same], ref["y"][same], f"{w.name} y")
+    if sample is None and differ == 0:
+        np.testing.assert_array_equal(counts, np.bincount(ref["topk_idx"].reshape(-1),
+                                                          minlength=w.E))
+    assert st.device_status() == 0
+    return st, near, differ
+
+
+def test_forward_tiny_whole_batch():
+    w, x, wt = _case(WORKLOADS["tiny"])
+    _forward_vs_oracle(w, x, wt)
+
+
+def test_forward_mid_sampled():
+    w, x, wt = _case(WORKLOADS["mid"])
+    _forward_vs_oracle(w, x, wt, sample=192)
+
+
+def test_forward_is_deterministic():
+    w, x, wt = _case(WORKLOADS["mid"], T=700)
+    st = Stages(w, x, wt)
+    st.forward()
+    y0 = st.y.clone()
+    c0 = st.counts.clone()
+    st.y.zero_()
+    st.forward()
+    assert torch.equal(st.y, y0) and torch.equal(st.counts, c0)
+
+
+def test_staged_calls_equal_forward():
+    w, x, wt = _case(WORKLOADS["mid"], T=333)
+    st = Stages(w, x, wt)
+    st.forward()
+    y_fwd = st.y.clone()
+    st.route()
+    st.dispatch()
+    check_dispatch_properties(to_np(st.topk_idx), to_np(st.counts), to_np(st.offsets),
+                              to_np(st.perm_tok), to_np(st.slot_pos), w.N, w.E)
+    st.expert_ffn()
+    st.combine()
+    assert torch.equal(st.y, y_fwd)
+
+
+# ---------------------------------------------------------------------------------- edge cases
+def test_zero_tokens():
+    w = Workload("t0", T=0, d=128, N=8, Z=4, K=3, I=256)
+    wt = make_weights(w)
+    x = torch.zeros((0, w.d), dtype=torch.bfloat16)
+    st = Stages(w, x, wt)
+    st.counts.fill_(5)
+    st.forward()
+    torch.cuda.synchronize()
+    assert (st.counts == 0).all()
+    assert st.device_status() == 0
+
+
+@pytest.mark.parametrize("T", [1, 77, 300])
+def test_ragged_token_counts(T):
+    w, x, wt = _case(WORKLOADS["tiny"], T=T, seed=T)
+    _forward_vs_oracle(w, x, wt)
+
+
+def test_all_zero_experts_return_sum_g_times_x():
+    w = WORKLOADS["tiny"]
+    b = torch.zeros(w.E)
+    b[w.N:] = 1.0
+    w, x, wt = _case(w, bias=b)
+    st = Stages(w, x, wt)
+    st.forward()
+    ref = oracle.router(x, wt["W_r"], b, w.K)
+    st.route()
+    assert (to_np(st.topk_idx) >= w.N).all()
+    assert (to_np(st.counts)[:w.N] == 0).all()
+    want = ref["topk_gate"].sum(axis=1, keepdims=True) * oracle.bf16_to_f64(oracle.bf16_bits(x))
+    assert_y_close(oracle.bf16_to_f64(to_np(st.y)), want, "zero-expert y")
+    assert st.device_status() == 0
+
+
+def test_one_expert_takes_every_token():
+    # Expert 3 is selected by all 1000 tokens: one group of 1000 rows spans 8 token tiles.
+    w = WORKLOADS["tiny"]
+    b = torch.zeros(w.E)
+    b[3] = 1.0
+    w, x, wt = _case(w, bias=b, T=1000, seed=2)
+    st, _, _ = _forward_vs_oracle(w, x, wt, sample=128)
+    assert to_np(st.counts)[3] == 1000
+
+
+def test_k_equals_all_experts():
+    w = Workload("all", T=96, d=128, N=8, Z=4, K=12, I=256, bias_range=0.0)
+    w, x, wt = _case(w)
+    st, _, _ = _forward_vs_oracle(w, x, wt)
+    st.route()
+    assert torch.isinf(st.gap).all()
+
+
+def test_widths_not_multiple_of_tiles():
+    # d = 192 (GEMM2 weight tile half-used), I = 320 (partial up-projection tile), E = 9.
+    w = Workload("odd", T=200, d=192, N=5, Z=4, K=3, I=320)
+    w, x, wt = _case(w, seed=4)
+    _forward_vs_oracle(w, x, wt)
+
+
+# ---------------------------------------------------------------------------------- error paths
+def test_device_status_codes():
+    w, x, wt = _case(WORKLOADS["tiny"])
+    st = Stages(w, x, wt)
+    st.offsets.copy_(torch.tensor([0, 5, 3, 9, 9, 9, 9, 9, 9], dtype=torch.int32))
+    st.y_perm.fill_(1.0)
+    st.expert_ffn()
+    assert st.device_status() == 0x300  # rows out of order: nothing computed, nothing faulted
+    assert (st.y_perm == 1.0).all()
+    assert st.device_status() == 0  # reading clears it
+    bad = torch.tensor([[0, 1, 99]] * w.T, dtype=torch.int32)
+    st.topk_idx.copy_(bad)
+    st.dispatch()
+    assert st.device_status() == 0x200  # expert id out of range, skipped
+    assert int(st.counts.sum()) == 2 * w.T
+
+
+def test_host_side_argument_errors():
+    w, x, wt = _case(WORKLOADS["tiny"])
+    st = Stages(w, x, wt)
+    with pytest.raises(mb.MoeError) as e:
+        mb.moe_forward(st.dm, st.x, wt["W_r"].to(DEV), wt["b"].to(DEV), wt["W_g"].to(DEV),
+                       wt["W_u"].to(DEV), wt["W_d"].to(DEV), st.y, st.counts, st.ws[:1024])
+    assert e.value.code == 4  # workspace too small
+    bad_dm = mb.dims(w.T, 100, w.N, w.Z, w.K, w.I)
+    assert mb.workspace_size(bad_dm) == 0

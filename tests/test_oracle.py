@@ -315,3 +315,27 @@ def test_brute_force_pin_catches_a_planted_sign_error():
         best = sorted(np.argsort(-s_lib[t], kind="stable")[:3].tolist())
         mismatches += r_bad["topk_idx"][t].tolist() != best
     assert mismatches > 0
+
+
+def test_combine_rows_agrees_with_whole_layer():
+    # Two routes to the same y: the whole layer, and dispatch + per-expert outputs + the
+    # weighted sum of given rows.  Both must agree with the single-expert library pin above.
+    w = WORKLOADS["tiny"]
+    wt = make_weights(w, seed=8)
+    x = make_tokens(w, seed=8)
+    b = (torch.rand(w.E, generator=torch.Generator().manual_seed(4)) * 0.02).float()
+    ref = oracle.forward(x, wt["W_r"], b, wt["W_g"], wt["W_u"], wt["W_d"], w.N, w.Z, w.K)
+    dsp = oracle.dispatch(ref["topk_idx"], w.N, w.E)
+    xb = oracle.bf16_bits(x)
+    rows = np.zeros((len(dsp["perm_tok"]), w.d))
+    gates = np.zeros(len(dsp["perm_tok"]))
+    for t in range(w.T):
+        for k in range(w.K):
+            if dsp["slot_pos"][t, k] >= 0:
+                gates[dsp["slot_pos"][t, k]] = ref["topk_gate"][t, k]
+    for e in range(w.N):
+        lo, hi = dsp["offsets"][e], dsp["offsets"][e + 1]
+        out = oracle.swiglu_expert(xb[dsp["perm_tok"][lo:hi]], wt["W_g"][e], wt["W_u"][e], wt["W_d"][e])
+        rows[lo:hi] = gates[lo:hi, None] * out
+    y = oracle.combine_rows(x, ref["topk_idx"], ref["topk_gate"], dsp["slot_pos"], rows, w.N)
+    np.testing.assert_allclose(y, ref["y"], rtol=1e-12, atol=1e-14)
