@@ -126,6 +126,24 @@ int moe_dispatch(const moe_dims *dims, const moe_bf16 *x, const int32_t *topk_id
                  float *perm_gate, int32_t *slot_pos, moe_bf16 *x_perm, void *ws,
                  size_t ws_bytes, void *stream);
 
+/* moe_dispatch for callers that cannot provide a workspace.  The pages have no counterpart;
+ * this exists for library users, not for the layer's definition.  Some callers cannot give
+ * the library device memory: a plugin whose host process owns all device memory through its
+ * own pool, or a deployment whose memory budget forbids allocations after start-up.  This
+ * variant takes the same arguments as moe_dispatch minus the workspace and produces the same
+ * outputs; its scratch is a fixed 1 MiB array inside the library image (present on every GPU
+ * that loads the library, until the process exits).
+ *   - needs ceil(T/256) * (N+Z) <= 262144; larger requests return MOE_ERR_WORKSPACE;
+ *   - calls share that array: two calls whose kernels overlap on the GPU race on it;
+ *   - device-side checks still skip bad accesses but have no status word to report to;
+ *   - the first call on a device looks up the array's device address with that device
+ *     current; make that first call before any stream capture.
+ * It allocates and frees nothing. */
+int moe_dispatch_noalloc(const moe_dims *dims, const moe_bf16 *x, const int32_t *topk_idx,
+                         const float *topk_gate, int32_t *counts, int32_t *offsets,
+                         int32_t *perm_tok, float *perm_gate, int32_t *slot_pos,
+                         moe_bf16 *x_perm, void *stream);
+
 /* The FFN experts on the grouped rows (grouped GEMMs on tcgen05 tensor cores):
  *   h[r]      = silu(x_perm[r] W_g[e]^T) * (x_perm[r] W_u[e]^T)       bf16 [T*K, I]
  *   y_perm[r] = perm_gate[r] * (h[r] W_d[e]^T)                          bf16 [T*K, d]

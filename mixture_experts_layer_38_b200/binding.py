@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 EXPORTS = (
     "moe_strerror", "moe_workspace_size", "moe_scratch_size", "moe_route", "moe_dispatch",
     "moe_expert_ffn", "moe_combine", "moe_bias_update", "moe_forward", "moe_forward_timed",
-    "moe_last_device_error",
+    "moe_last_device_error", "moe_dispatch_noalloc",
 )
 NUM_STAGE_EVENTS = 7
 STAGE_NAMES = ("router_gemm", "route_topk", "dispatch", "ffn_up_gemm", "ffn_down_gemm",
@@ -77,9 +77,10 @@ def lib():
         L.moe_forward_timed.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S,
                                         ctypes.POINTER(ctypes.c_void_p), _P]
         L.moe_last_device_error.argtypes = [_P, _P]
+        L.moe_dispatch_noalloc.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
         for f in ("moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine",
                   "moe_bias_update", "moe_forward", "moe_forward_timed",
-                  "moe_last_device_error"):
+                  "moe_last_device_error", "moe_dispatch_noalloc"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -167,6 +168,22 @@ def moe_dispatch(dm, x, topk_idx, topk_gate, counts, offsets, perm_tok, perm_gat
         _ptr(slot_pos, torch.int32, (dm.T, dm.K), "slot_pos"),
         _ptr(x_perm, torch.bfloat16, (R, dm.d), "x_perm"), w, n, _stream(stream))
     _check("moe_dispatch", rc)
+
+
+def moe_dispatch_noalloc(dm, x, topk_idx, topk_gate, counts, offsets, perm_tok, perm_gate,
+                         slot_pos, x_perm, stream=None):
+    """moe_dispatch without a workspace, for callers that cannot hand the library device
+    memory; its scratch is a fixed array inside the library (see include/moe.h)."""
+    E, R = dm.N + dm.Z, dm.T * dm.K
+    rc = lib().moe_dispatch_noalloc(
+        ctypes.byref(dm), _ptr(x, torch.bfloat16, (dm.T, dm.d), "x"),
+        _ptr(topk_idx, torch.int32, (dm.T, dm.K), "topk_idx"),
+        _ptr(topk_gate, torch.float32, (dm.T, dm.K), "topk_gate"),
+        _ptr(counts, torch.int32, (E,), "counts"), _ptr(offsets, torch.int32, (dm.N + 1,), "offsets"),
+        _ptr(perm_tok, torch.int32, (R,), "perm_tok"), _ptr(perm_gate, torch.float32, (R,), "perm_gate"),
+        _ptr(slot_pos, torch.int32, (dm.T, dm.K), "slot_pos"),
+        _ptr(x_perm, torch.bfloat16, (R, dm.d), "x_perm"), _stream(stream))
+    _check("moe_dispatch_noalloc", rc)
 
 
 def moe_expert_ffn(dm, x_perm, offsets, perm_gate, W_g, W_u, W_d, h, y_perm, ws, stream=None):
