@@ -21,8 +21,11 @@
 //   warp 1      TMEM allocator (512 columns = 2 buffers x 2 accumulators x 128) and MMA issuer
 //   warps 2-5   epilogue: tcgen05.ld from TMEM, fused SwiGLU / gate scaling / fp32 store via a
 //               per-warp shared-memory transpose and coalesced row stores
-// Tiles are ordered by group, then token tile, then weight tile, so CTAs running at the same
-// time share the token tile and walk one expert's weights together (L2 reuse).
+// Token tiles come in two kinds: full 128-row tiles (compute-bound) and each expert's partial
+// tail tile (for the many lightly loaded experts: weight streaming).  The static schedule
+// interleaves the two lists in proportion, and within a token tile the weight tiles come
+// fastest, so the CTAs in flight share token tiles and walk one expert's weights together (L2
+// reuse) while the tensor cores and HBM stay busy at the same time.
 //
 // Every wait is bounded (device.cuh): on timeout the kernel records MOE_DEV_WAIT_TIMEOUT, all
 // roles unwind, in-flight copies and MMAs are drained (again bounded) and TMEM is freed.
@@ -47,7 +50,7 @@ constexpr long long kDrainLimitCycles = 1ll << 30;
 
 constexpr int kSmemStages = kStages * kStageBytes;
 constexpr int kSmemStaging = kEpiWarps * kStagingFloats * 4;
-constexpr int kSmemPrefix = (kMaxGroups + 4) * 4;
+constexpr int kSmemPrefix = 2 * (kMaxGroups + 4) * 4;  // full-tile and tail-tile prefixes
 constexpr int kNumBars = 2 * kStages + 4 + 1;
 constexpr int kSmemBytes = 1024 + kSmemStages + kSmemStaging + kSmemPrefix + kNumBars * 8 + 16;
 
@@ -63,9 +66,16 @@ struct Tile {
   int split;
 };
 
+// Token tiles of a group (expert) with c rows: floor(c/128) full 128-row tiles ("heavy":
+// compute-bound at d = 6144) and, if c % 128 != 0, one partial tail tile ("light": for the many
+// experts with a handful of tokens it only streams the expert's weights).  The schedule merges
+// the two lists so the tiles in flight at any moment mix both kinds and the tensor cores and
+// HBM are busy together: of the first p+1 merged positions, floor((p+1) L / (H+L)) are light.
 struct Schedule {
-  const int *prefix;  // [G + 1] token-tile prefix per group (shared memory)
+  const int *hpre;  // [G + 1] prefix of full tiles per group (shared memory)
+  const int *lpre;  // [G + 1] prefix of tail tiles per group
   int G;
+  int H, L;         // total full / tail tiles
   int m_tiles;
   int splits;
   int total;
@@ -76,23 +86,38 @@ __device__ __forceinline__ int group_off(const GemmArgs &a, int g) {
   return __ldg(a.group_offsets + g);
 }
 
+// Largest g in [0, G) with pre[g] <= v (pre non-decreasing, pre[0] = 0 <= v).
+__device__ __forceinline__ int find_group(const int *pre, int G, int v) {
+  int lo = 0, hi = G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (pre[mid] <= v) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
 template <int EPI>
 __device__ __forceinline__ Tile decode_tile(const GemmArgs &a, const Schedule &s, int tile) {
   Tile t;
   const int mt = tile % s.m_tiles;
   const int rest = tile / s.m_tiles;
   t.split = rest % s.splits;
-  const int ntg = rest / s.splits;
-  int lo = 0, hi = s.G - 1;  // largest g with prefix[g] <= ntg
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (s.prefix[mid] <= ntg) lo = mid; else hi = mid - 1;
+  const int pos = rest / s.splits;
+  const long long P = (long long)s.H + s.L;
+  const int light_upto = (int)(((long long)pos + 1) * s.L / P);
+  const int light_before = (int)((long long)pos * s.L / P);
+  int g;
+  if (light_upto > light_before) {  // the (light_upto-1)-th tail tile
+    g = find_group(s.lpre, s.G, light_upto - 1);
+    const int lo = group_off(a, g), hi = group_off(a, g + 1);
+    t.row0 = lo + ((hi - lo) / kBN) * kBN;
+    t.n_valid = hi - t.row0;
+  } else {  // the (pos - light_before)-th full tile
+    const int i = pos - light_before;
+    g = find_group(s.hpre, s.G, i);
+    t.row0 = group_off(a, g) + (i - s.hpre[g]) * kBN;
+    t.n_valid = kBN;
   }
-  const int g = lo;
-  const int nt = ntg - s.prefix[g];
-  const int g_end = group_off(a, g + 1);
-  t.row0 = group_off(a, g) + nt * kBN;
-  t.n_valid = min(kBN, g_end - t.row0);
   t.nb = (t.n_valid + 15) & ~15;
   if (EPI == kEpiSwiGLU) {
     t.m0 = mt * kBM;
@@ -111,45 +136,68 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs &a, const Schedule &s
   return t;
 }
 
-// Token-tile prefix over groups, computed by all threads of the block.  Returns false (and
-// records MOE_DEV_BAD_ROWS) if the offsets are not monotone or exceed the activation rows.
-__device__ bool build_schedule(const GemmArgs &a, int *prefix, int *scratch, Schedule &s) {
-  const int G = a.group_offsets ? a.num_groups : 1;
-  const int per = (G + kGemmThreads - 1) / kGemmThreads;
-  const int g_begin = min(G, (int)threadIdx.x * per);
-  const int g_end = min(G, g_begin + per);
-  int local = 0;
-  bool bad = false;
-  for (int g = g_begin; g < g_end; ++g) {
-    const int lo = group_off(a, g), hi = group_off(a, g + 1);
-    if (lo < 0 || hi < lo || hi > a.rows) { bad = true; continue; }
-    local += (hi - lo + kBN - 1) / kBN;
-  }
+// Exclusive block-wide scan of one int per thread; returns the thread's exclusive prefix and
+// the block total.  `scratch` holds one int per warp.
+__device__ __forceinline__ int block_exclusive_scan(int v, int *scratch, int &total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = local;
+  int incl = v;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += v;
+    const int o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
   }
   if (lane == 31) scratch[warp] = incl;
   __syncthreads();
   int base = 0;
-  for (int w = 0; w < warp; ++w) base += scratch[w];
-  int run = base + incl - local;
-  for (int g = g_begin; g < g_end; ++g) {
-    prefix[g] = run;
-    const int lo = group_off(a, g), hi = group_off(a, g + 1);
-    if (!(lo < 0 || hi < lo || hi > a.rows)) run += (hi - lo + kBN - 1) / kBN;
+  total = 0;
+  for (int w = 0; w < kGemmThreads / 32; ++w) {
+    if (w < warp) base += scratch[w];
+    total += scratch[w];
   }
-  int total = 0;
-  for (int w = 0; w < kGemmThreads / 32; ++w) total += scratch[w];
-  if (threadIdx.x == 0) prefix[G] = total;
+  __syncthreads();
+  return base + incl - v;
+}
+
+// Full-tile and tail-tile prefixes over groups, computed by all threads of the block.  Returns
+// false (and records MOE_DEV_BAD_ROWS) if the offsets are not monotone or exceed the rows.
+__device__ bool build_schedule(const GemmArgs &a, int *hpre, int *lpre, int *scratch,
+                               Schedule &s) {
+  const int G = a.group_offsets ? a.num_groups : 1;
+  const int per = (G + kGemmThreads - 1) / kGemmThreads;
+  const int g_begin = min(G, (int)threadIdx.x * per);
+  const int g_end = min(G, g_begin + per);
+  int nh = 0, nl = 0;
+  bool bad = false;
+  for (int g = g_begin; g < g_end; ++g) {
+    const int lo = group_off(a, g), hi = group_off(a, g + 1);
+    if (lo < 0 || hi < lo || hi > a.rows) { bad = true; continue; }
+    nh += (hi - lo) / kBN;
+    nl += ((hi - lo) % kBN) != 0;
+  }
+  int H = 0, L = 0;
+  int hrun = block_exclusive_scan(nh, scratch, H);
+  int lrun = block_exclusive_scan(nl, scratch, L);
+  for (int g = g_begin; g < g_end; ++g) {
+    hpre[g] = hrun;
+    lpre[g] = lrun;
+    const int lo = group_off(a, g), hi = group_off(a, g + 1);
+    if (!(lo < 0 || hi < lo || hi > a.rows)) {
+      hrun += (hi - lo) / kBN;
+      lrun += ((hi - lo) % kBN) != 0;
+    }
+  }
+  if (threadIdx.x == 0) {
+    hpre[G] = H;
+    lpre[G] = L;
+  }
   const bool any_bad = __syncthreads_or(bad);
   if (any_bad && threadIdx.x == 0) record_status(a.status, MOE_DEV_BAD_ROWS);
-  s.prefix = prefix;
+  s.hpre = hpre;
+  s.lpre = lpre;
   s.G = G;
-  s.total = any_bad ? 0 : total;
+  s.H = any_bad ? 0 : H;
+  s.L = any_bad ? 0 : L;
+  s.total = s.H + s.L;  // token tiles; times m_tiles and splits by the caller
   return !any_bad;
 }
 
@@ -266,7 +314,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t *ring = smem;
   float *staging = reinterpret_cast<float *>(smem + kSmemStages);
-  int *prefix = reinterpret_cast<int *>(smem + kSmemStages + kSmemStaging);
+  int *hpre = reinterpret_cast<int *>(smem + kSmemStages + kSmemStaging);
+  int *lpre = hpre + kMaxGroups + 4;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kSmemStages + kSmemStaging + kSmemPrefix);
   uint64_t *full_bar = bars;
   uint64_t *empty_bar = bars + kStages;
@@ -303,7 +352,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tmem_relinquish();
   }
   Schedule sched;
-  build_schedule(args, prefix, reinterpret_cast<int *>(staging), sched);
+  build_schedule(args, hpre, lpre, reinterpret_cast<int *>(staging), sched);
   sched.m_tiles = m_tiles_of<EPI>(args.M);
   sched.splits = EPI == kEpiF32 ? args.k_splits : 1;
   sched.total = sched.total * sched.m_tiles * sched.splits;

@@ -15,6 +15,8 @@ Z zero-computation experts, K experts per token):
 
 The expert pool size (512 FFN + 256 zero experts, K=12) and the ~8 activated experts follow
 the LongCat-Flash descriptions ("美团LongCat-Flash：算力调度新纪元", §技术创新, caption (b)).
+``pid_target`` is the set-point of the PID step the benchmark runs after every forward pass:
+8 FFN experts per token at K=12, and the same 2/3 share of K for the small workloads.
 
 Distributions: x ~ N(0, 1) and every weight ~ N(0, 0.02^2), rounded to bf16; biases fp32.
 Weights come from one generator seeded with ``seed`` in the order W_r, b, then per expert
@@ -66,8 +68,8 @@ class Workload:
 
 
 WORKLOADS = {
-    "tiny": Workload("tiny", T=64, d=128, N=8, Z=4, K=3, I=256, bias_range=0.0),
-    "mid": Workload("mid", T=4096, d=2048, N=64, Z=32, K=6, I=1024),
+    "tiny": Workload("tiny", T=64, d=128, N=8, Z=4, K=3, I=256, bias_range=0.0, pid_target=2.0),
+    "mid": Workload("mid", T=4096, d=2048, N=64, Z=32, K=6, I=1024, pid_target=4.0),
     "decode": Workload("decode", T=128, d=6144, N=512, Z=256, K=12, I=2048),
     "prefill": Workload("prefill", T=16384, d=6144, N=512, Z=256, K=12, I=2048),
     "skewed": Workload("skewed", T=8192, d=6144, N=512, Z=256, K=12, I=2048, zipf_s=1.1,
