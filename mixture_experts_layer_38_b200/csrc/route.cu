@@ -1,4 +1,4 @@
-// route.cu -- softmax router R and biased top-K selection, one warp per token.
+// route.cu -- softmax router R and biased top-K selection, one thread block per token.
 //
 // "衝上熱搜！美團大模型，靠「快」火了", §零計算專家: R is a softmax router over the N FFN experts
 // and Z zero-computation experts; a per-expert bias b_i adjusts the routing score used to pick
@@ -7,9 +7,10 @@
 //   p   = exp(l - max l) / sum exp(l - max l)
 //   s   = p + b;  the K largest s are selected, an exact tie going to the lower expert id
 //   out = selected ids in ascending order, gates g = p (not renormalised), gap = s_(K) - s_(K+1)
-// Lane j holds experts j, j+32, j+64, ... in registers; each of the K+1 selection rounds is a
-// local scan plus a 5-step butterfly argmax over (score desc, id asc), so the result does not
-// depend on thread timing.
+// Thread i of the 256-thread block holds experts i, i+256, i+512, i+768 in registers, so the
+// split-K partial sums, exp and bias are spread over 8 warps; each of the K+1 selection rounds
+// is a block-wide argmax of one 64-bit key per thread, and the result does not depend on
+// thread timing.
 #include <math.h>
 
 #include "device.cuh"
@@ -18,32 +19,57 @@
 namespace moe {
 namespace {
 
-constexpr int kRouteWarps = 8;
+// Selection key of expert id with score s:
+// (order-preserving bits of s) << 32 | (0xffffffff - id)  ->  larger score, then lower id.
+constexpr int kBlockThreads = 256;
+constexpr int kPerThread = 4;  // E <= 1024
 
-struct Cand {
-  float s;  // biased score
-  float p;  // router probability
-  int id;
-};
-
-__device__ __forceinline__ bool better(const Cand &a, const Cand &b) {
-  return a.s > b.s || (a.s == b.s && a.id < b.id);
+__device__ __forceinline__ uint64_t score_key(float s, int id) {
+  uint32_t u = __float_as_uint(s);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return (static_cast<uint64_t>(u) << 32) | (0xffffffffu - static_cast<uint32_t>(id));
 }
 
-template <int PER>
-__global__ void __launch_bounds__(kRouteWarps * 32)
-    route_topk_kernel(const float *__restrict__ logits, int splits, int T, int E, int ld, int K,
-                      const float *__restrict__ b, int32_t *__restrict__ topk_idx,
-                      float *__restrict__ topk_gate, float *__restrict__ gap, int *status) {
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * kRouteWarps + (threadIdx.x >> 5);
-  if (t >= T) return;
-  const long long split_stride = (long long)T * ld;
-
-  float l[PER];
+__device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
 #pragma unroll
-  for (int j = 0; j < PER; ++j) {
-    const int e = lane + 32 * j;
+  for (int off = 16; off > 0; off >>= 1) {
+    const uint64_t o = __shfl_xor_sync(0xffffffffu, v, off);
+    v = o > v ? o : v;
+  }
+  return v;
+}
+
+__device__ __forceinline__ float block_reduce(float v, bool is_max, float *red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float o = __shfl_xor_sync(0xffffffffu, v, off);
+    v = is_max ? fmaxf(v, o) : v + o;
+  }
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float r = red[0];
+  for (int w = 1; w < kBlockThreads / 32; ++w) r = is_max ? fmaxf(r, red[w]) : r + red[w];
+  __syncthreads();
+  return r;
+}
+
+__global__ void __launch_bounds__(kBlockThreads)
+    route_topk_block_kernel(const float *__restrict__ logits, int splits, int T, int E, int ld,
+                            int K, const float *__restrict__ b, int32_t *__restrict__ topk_idx,
+                            float *__restrict__ topk_gate, float *__restrict__ gap, int *status) {
+  __shared__ float red[kBlockThreads / 32];
+  __shared__ uint64_t wbest[kBlockThreads / 32];
+  __shared__ int sel_id[33];
+  __shared__ float sel_p[33];
+  __shared__ float sel_s[33];
+  const int t = blockIdx.x;
+  const int tid = threadIdx.x;
+  const long long split_stride = (long long)T * ld;
+  float l[kPerThread];
+#pragma unroll
+  for (int j = 0; j < kPerThread; ++j) {
+    const int e = tid + kBlockThreads * j;
     float v = -INFINITY;
     if (e < E) {
       const float *src = logits + (long long)t * ld + e;
@@ -52,78 +78,71 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
     }
     l[j] = v;
   }
-  float m = -INFINITY;
+  float m = l[0];
 #pragma unroll
-  for (int j = 0; j < PER; ++j) m = fmaxf(m, l[j]);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  for (int j = 1; j < kPerThread; ++j) m = fmaxf(m, l[j]);
+  m = block_reduce(m, true, red);
   float z = 0.f;
 #pragma unroll
-  for (int j = 0; j < PER; ++j) {
-    const int e = lane + 32 * j;
-    l[j] = (e < E) ? expf(l[j] - m) : 0.f;  // l now holds exp(l - max)
+  for (int j = 0; j < kPerThread; ++j) {
+    const int e = tid + kBlockThreads * j;
+    l[j] = (e < E) ? expf(l[j] - m) : 0.f;  // now exp(l - max)
     z += l[j];
   }
+  z = block_reduce(z, false, red);
+  float p[kPerThread];
+  uint64_t key[kPerThread];
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
-
-  float p[PER], s[PER];
-#pragma unroll
-  for (int j = 0; j < PER; ++j) {
-    const int e = lane + 32 * j;
+  for (int j = 0; j < kPerThread; ++j) {
+    const int e = tid + kBlockThreads * j;
     p[j] = __fdiv_rn(l[j], z);
-    s[j] = (e < E) ? __fadd_rn(p[j], __ldg(b + e)) : -INFINITY;
+    key[j] = (e < E) ? score_key(__fadd_rn(p[j], __ldg(b + e)), e) : 0ull;
   }
-
-  uint32_t chosen = 0;
-  int my_id = 0x7fffffff;  // lane k (< K) keeps the k-th selected expert
-  float my_gate = 0.f;
-  float kth = INFINITY, next = -INFINITY;
-  for (int k = 0; k <= K && k < E; ++k) {
-    Cand c{-INFINITY, 0.f, 0x7fffffff};
+  const int rounds = K < E ? K + 1 : K;
+  for (int k = 0; k < rounds; ++k) {
+    uint64_t best = key[0];
 #pragma unroll
-    for (int j = 0; j < PER; ++j) {
-      const int e = lane + 32 * j;
-      const Cand o{s[j], p[j], e};
-      if (e < E && !((chosen >> j) & 1u) && (c.id == 0x7fffffff || better(o, c))) c = o;
-    }
+    for (int j = 1; j < kPerThread; ++j) best = key[j] > best ? key[j] : best;
+    best = warp_max_u64(best);
+    if ((tid & 31) == 0) wbest[tid >> 5] = best;
+    __syncthreads();
+    uint64_t win = wbest[0];
+    for (int w = 1; w < kBlockThreads / 32; ++w) win = wbest[w] > win ? wbest[w] : win;
+    const int id = (int)(0xffffffffu - (uint32_t)(win & 0xffffffffu));
+    if (win == 0ull) {  // nothing left that is selectable (non-finite scores): flag, skip
+      if (tid == 0) {
+        record_status(status, MOE_DEV_BAD_EXPERT);
+        sel_id[k] = 0x7fffffff;
+      }
+    } else if (id % kBlockThreads == tid) {
+      const int j = id / kBlockThreads;
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      Cand o;
-      o.s = __shfl_xor_sync(0xffffffffu, c.s, off);
-      o.p = __shfl_xor_sync(0xffffffffu, c.p, off);
-      o.id = __shfl_xor_sync(0xffffffffu, c.id, off);
-      if (o.id != 0x7fffffff && (c.id == 0x7fffffff || better(o, c))) c = o;
+      for (int jj = 0; jj < kPerThread; ++jj) {
+        if (jj == j) {
+          sel_id[k] = id;
+          sel_p[k] = p[jj];
+          sel_s[k] = __fadd_rn(p[jj], __ldg(b + id));
+          key[jj] = 0ull;
+        }
+      }
     }
-    if (c.id == 0x7fffffff) {  // only non-finite scores were left: flag, never index with it
-      if (lane == 0) record_status(status, MOE_DEV_BAD_EXPERT);
-      break;
+    __syncthreads();
+  }
+  if (tid < 32) {
+    const int lane = tid;
+    const int my_id = lane < K ? sel_id[lane] : 0x7fffffff;
+    int rank = 0;
+    for (int k2 = 0; k2 < K; ++k2) {
+      const int other = __shfl_sync(0xffffffffu, my_id, k2);
+      rank += other < my_id;
     }
-    if (k == K) { next = c.s; break; }
-    if (lane == (c.id & 31)) chosen |= 1u << (c.id >> 5);
-    if (lane == k) { my_id = c.id; my_gate = c.p; }
-    kth = c.s;
+    if (lane < K) {
+      topk_idx[(long long)t * K + rank] = my_id;
+      topk_gate[(long long)t * K + rank] = sel_p[lane];
+    }
+    if (gap != nullptr && lane == 0)
+      gap[t] = (K < E) ? __fsub_rn(sel_s[K - 1], sel_s[K]) : INFINITY;
   }
-
-  // Ascending-id order: rank of my id among the K selected ids (all distinct).
-  int rank = 0;
-  for (int k2 = 0; k2 < K; ++k2) {
-    const int other = __shfl_sync(0xffffffffu, my_id, k2);
-    rank += other < my_id;
-  }
-  if (lane < K) {
-    topk_idx[(long long)t * K + rank] = my_id;
-    topk_gate[(long long)t * K + rank] = my_gate;
-  }
-  if (gap != nullptr && lane == 0) gap[t] = (K < E) ? __fsub_rn(kth, next) : INFINITY;
-}
-
-template <int PER>
-void launch_per(const float *logits, int splits, int T, int E, int ld, int K, const float *b,
-                int32_t *idx, float *gate, float *gap, int *status, cudaStream_t stream) {
-  const int grid = (T + kRouteWarps - 1) / kRouteWarps;
-  route_topk_kernel<PER><<<grid, kRouteWarps * 32, 0, stream>>>(logits, splits, T, E, ld, K, b,
-                                                                 idx, gate, gap, status);
 }
 
 }  // namespace
@@ -133,14 +152,8 @@ cudaError_t launch_route_topk(const float *logits, int splits, int T, int E, int
                               int *status, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
   const int ld = (E + 3) & ~3;
-  const int per = (E + 31) / 32;
-  if (per <= 1) launch_per<1>(logits, splits, T, E, ld, K, b, topk_idx, topk_gate, gap, status, stream);
-  else if (per <= 2) launch_per<2>(logits, splits, T, E, ld, K, b, topk_idx, topk_gate, gap, status, stream);
-  else if (per <= 4) launch_per<4>(logits, splits, T, E, ld, K, b, topk_idx, topk_gate, gap, status, stream);
-  else if (per <= 8) launch_per<8>(logits, splits, T, E, ld, K, b, topk_idx, topk_gate, gap, status, stream);
-  else if (per <= 16) launch_per<16>(logits, splits, T, E, ld, K, b, topk_idx, topk_gate, gap, status, stream);
-  else if (per <= 24) launch_per<24>(logits, splits, T, E, ld, K, b, topk_idx, topk_gate, gap, status, stream);
-  else launch_per<32>(logits, splits, T, E, ld, K, b, topk_idx, topk_gate, gap, status, stream);
+  route_topk_block_kernel<<<T, kBlockThreads, 0, stream>>>(logits, splits, T, E, ld, K, b,
+                                                          topk_idx, topk_gate, gap, status);
   return cudaGetLastError();
 }
 
