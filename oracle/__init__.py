@@ -42,9 +42,11 @@ def _load():
                                              _ptr, _ptr]
         _lib.oracle_pid_step.argtypes = [_i64, _i64, _i64, _ptr, _ptr, _ptr, ctypes.c_float,
                                          ctypes.c_float, ctypes.c_float, ctypes.c_float]
+        _lib.oracle_renormalize_gates.argtypes = [_i64, _i64, _ptr]
+        _lib.oracle_balance_step.argtypes = [_i64, _ptr, _ptr, ctypes.c_float]
         for f in ("oracle_router", "oracle_dispatch", "oracle_swiglu_expert",
                   "oracle_combine_tokens", "oracle_combine_rows", "oracle_forward",
-                  "oracle_pid_step"):
+                  "oracle_pid_step", "oracle_renormalize_gates", "oracle_balance_step"):
             getattr(_lib, f).restype = None
     return _lib
 
@@ -83,12 +85,13 @@ def bf16_to_f64(bits):
     return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
-def router(x, W_r, b, K, want_probs=False, want_scores=False):
+def router(x, W_r, b, K, want_probs=False, want_scores=False, renormalize=False):
     """Softmax router R and biased top-K (P1 §零計算專家).
 
     x: [T, d] bf16, W_r: [E, d] bf16, b: [E] fp32.  Returns a dict with ``topk_idx`` [T, K]
-    int32 in ascending expert id, ``topk_gate`` [T, K] fp64 (= p_i, not renormalised),
-    ``gap`` [T] fp64 (= s_(K) - s_(K+1)), and optionally ``probs`` / ``scores`` [T, E] fp64.
+    int32 in ascending expert id, ``topk_gate`` [T, K] fp64 (= p_i, not renormalised unless
+    ``renormalize``: then p_i over the sum of the K selected p), ``gap`` [T] fp64
+    (= s_(K) - s_(K+1)), and optionally ``probs`` / ``scores`` [T, E] fp64.
     """
     x, W_r, b = bf16_bits(x), bf16_bits(W_r), _f32(b)
     T, d = x.shape
@@ -104,7 +107,17 @@ def router(x, W_r, b, K, want_probs=False, want_scores=False):
     _load().oracle_router(T, d, E, K, _p(x), _p(W_r), _p(b), _p(out["topk_idx"]),
                           _p(out["topk_gate"]), _p(out["gap"]), _p(out["probs"]),
                           _p(out["scores"]))
+    if renormalize:
+        renormalize_gates(out["topk_gate"])
     return out
+
+
+def renormalize_gates(topk_gate):
+    """In place: each token's K gates divided by their sum (the renormalised-gate variant)."""
+    assert topk_gate.dtype == np.float64 and topk_gate.flags.c_contiguous
+    T, K = topk_gate.shape
+    _load().oracle_renormalize_gates(T, K, _p(topk_gate))
+    return topk_gate
 
 
 def dispatch(topk_idx, N, E):
@@ -166,13 +179,19 @@ def combine_rows(x, topk_idx, topk_gate, slot_pos, rows, N):
     return y
 
 
-def forward(x, W_r, b, W_g, W_u, W_d, N, Z, K):
-    """The whole layer for every token: router, biased top-K, experts, weighted sum (fp64)."""
+def forward(x, W_r, b, W_g, W_u, W_d, N, Z, K, renormalize=False):
+    """The whole layer for every token: router, biased top-K, experts, weighted sum (fp64).
+
+    With ``renormalize`` the gates are renormalised over the selected set before the sum."""
     x, W_r, b = bf16_bits(x), bf16_bits(W_r), _f32(b)
     W_g, W_u, W_d = bf16_bits(W_g), bf16_bits(W_u), bf16_bits(W_d)
     T, d = x.shape
     I = W_g.shape[1]
     assert W_r.shape == (N + Z, d) and W_g.shape == (N, I, d) and W_d.shape == (N, d, I)
+    if renormalize:
+        r = router(x, W_r, b, K, renormalize=True)
+        y = combine_tokens(np.arange(T), x, r["topk_idx"], r["topk_gate"], W_g, W_u, W_d, N)
+        return {"y": y, "topk_idx": r["topk_idx"], "topk_gate": r["topk_gate"], "gap": r["gap"]}
     y = np.zeros((T, d), np.float64)
     idx = np.zeros((T, K), np.int32)
     gate = np.zeros((T, K), np.float64)
@@ -221,3 +240,12 @@ def pid_step(counts, b, state, N, K, T, target, kp, ki, kd):
     assert b.dtype == np.float32 and b.flags.c_contiguous
     assert state.dtype == np.float32 and state.shape == (2,)
     _load().oracle_pid_step(N, K, T, _p(counts), _p(b), _p(state), target, kp, ki, kd)
+
+
+def balance_step(counts, b, N, gamma):
+    """Per-expert balancing term, in place: b_i += gamma * sign(mean FFN load - counts_i), i < N.
+
+    b: float32 [E] numpy array.  Applied after :func:`pid_step` when both are used."""
+    counts = _i32(counts)
+    assert b.dtype == np.float32 and b.flags.c_contiguous
+    _load().oracle_balance_step(N, _p(counts), _p(b), gamma)

@@ -317,3 +317,45 @@ void oracle_pid_step(int64_t N, int64_t K, int64_t T, const int32_t *counts, flo
     state[1] = e;
     for (int64_t i = 0; i < N; ++i) b[i] = b[i] + u;
 }
+
+/* ------------------------------------------------------------------------------------------
+ * Gate renormalisation over the selected set (an optional variant; the layer's default keeps
+ * the unrenormalised softmax gate, P1 §零計算專家).  Per token t:
+ *
+ *   g_k = g_k / sum_{j < K} g_j        (fp64, sum in slot order)
+ *
+ * The sum runs over all K selected experts, zero-computation ones included, so the weights
+ * of every y_t term (identity terms too) add up to one.
+ * ---------------------------------------------------------------------------------------- */
+void oracle_renormalize_gates(int64_t T, int64_t K, double *topk_gate)
+{
+    for (int64_t t = 0; t < T; ++t) {
+        double sum = 0.0;
+        for (int64_t k = 0; k < K; ++k) sum += topk_gate[t * K + k];
+        for (int64_t k = 0; k < K; ++k) topk_gate[t * K + k] = topk_gate[t * K + k] / sum;
+    }
+}
+
+/* ------------------------------------------------------------------------------------------
+ * Per-expert balancing term of the aux-loss-free bias scheme that the PID controller
+ * modifies (P1 §零計算專家: the expert-specific bias is adjusted from recent expert usage).
+ * The pages name the scheme without its rule; this is its published form: after a step,
+ * every FFN expert's bias moves by a fixed amount gamma toward the mean load,
+ *
+ *   c_mean = (sum_{i<N} counts_i) / N
+ *   b_i    = b_i + gamma * sign(c_mean - counts_i)     for i < N   (sign(0) = 0)
+ *
+ * The sign is taken exactly, from the integers: sign(c_mean - c_i) = sign(total - N*c_i).
+ * gamma * (+1 | 0 | -1) is exact, so the only rounding is the fp32 add.  Zero-expert biases
+ * are unchanged.  When combined with the PID step, the PID step is applied first.
+ * ---------------------------------------------------------------------------------------- */
+void oracle_balance_step(int64_t N, const int32_t *counts, float *b, float gamma)
+{
+    int64_t total = 0;
+    for (int64_t i = 0; i < N; ++i) total += counts[i];
+    for (int64_t i = 0; i < N; ++i) {
+        const int64_t diff = total - N * (int64_t)counts[i];
+        const float s = diff > 0 ? 1.0f : (diff < 0 ? -1.0f : 0.0f);
+        b[i] = b[i] + gamma * s;
+    }
+}
