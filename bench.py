@@ -36,6 +36,8 @@ from mixture_experts_layer_38_b200.workloads import WORKLOADS, make_tokens, make
 
 METRIC = "MoE-layer tokens/s"
 UNIT = "tokens/s"
+NOMINAL_BF16_TFLOPS = 2250.0  # B200 dense bf16 datasheet figure
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e datasheet figure
 PID_GAINS = (0.005, 0.002, 0.0)  # kp, ki, kd
 LAUNCHES_PER_STEP = 10  # router GEMM, top-K, histogram, scan, permute, gather, 2 GEMMs,
                         # combine, PID
@@ -43,7 +45,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic per launch of the dominant kernel from an ncu capture (profiles/), valid only
 # while the kernel source is unchanged (sha1 of the GEMM source at capture time).
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    ("prefill", "ffn_up_gemm"): {"bytes_per_launch": 41_834_767_616, "src": "44b67aaf0a11"},
+    ("decode", "ffn_up_gemm"): {"bytes_per_launch": 7_316_203_008, "src": "44b67aaf0a11"},
+}
 
 
 def log(*a):
@@ -61,7 +66,7 @@ def peaks():
 
 def gemm_source_hash():
     h = hashlib.sha1()
-    for name in ("gemm.cu", "device.cuh"):
+    for name in ("gemm.cu", "device.cuh", "kernels.cuh"):
         with open(os.path.join(ROOT, "mixture_experts_layer_38_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:12]
@@ -84,64 +89,111 @@ def job_throughput(world: int, tokens_per_rank: int, steps: int, ms: float) -> f
 
 # ------------------------------------------------------------------------------ clocks
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock, power and clock-event reasons sampled DURING the timed region (read-only).
+
+    NVML (the library nvidia-smi reads) polled every 10 ms from a thread, so even a timed region
+    of a few hundred ms yields dozens of samples; nvidia-smi's loop mode is the fallback."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
+    SMI_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device):
-        self.proc = None
-        self.path = None
+        self.uuid = None
         try:
-            uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+            self.uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
         except Exception:
-            uuid = str(device)
-        self.gpu = uuid
+            pass
+        self.samples = []
+        self.max_mhz = None
+        self.power_limit_w = None
+        self._stop = None
+        self._thread = None
+        self._proc = None
+        self._path = None
+        self.source = None
 
     def start(self):
-        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        import threading
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByUUID(self.uuid) if self.uuid else \
+                pynvml.nvmlDeviceGetHandleByIndex(torch.cuda.current_device())
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            try:
+                self.power_limit_w = pynvml.nvmlDeviceGetEnforcedPowerLimit(h) / 1000.0
+            except Exception:
+                pass
+            bits = [(name, getattr(pynvml, const)) for name, const in self.REASONS]
+            self._stop = threading.Event()
+
+            def loop():
+                while not self._stop.is_set():
+                    try:
+                        mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                        watts = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
+                        r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.samples.append((mhz, watts, [n for n, bit in bits if r & bit]))
+                    except Exception:
+                        pass
+                    self._stop.wait(0.01)
+            self._thread = threading.Thread(target=loop, daemon=True)
+            self._thread.start()
+            self.source = "nvml 10 ms"
+            return
+        except Exception as e:
+            log("NVML clock sampling unavailable, falling back to nvidia-smi:", e)
+        fd, self._path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", self.gpu, f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except Exception as e:  # nvidia-smi missing: report no clocks
+            self._proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.uuid or "0", f"--query-gpu={self.SMI_FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self._path, "w"), stderr=subprocess.DEVNULL)
+            self.source = "nvidia-smi 100 ms"
+        except Exception as e:
             log("clock sampling unavailable:", e)
-            self.proc = None
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        time.sleep(0.25)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-
-        def num(v):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=2)
+        elif self._proc is not None:
+            time.sleep(0.15)
+            self._proc.terminate()
             try:
-                return float(v)
-            except ValueError:
-                return None
-        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
-        smax = [num(r[2]) for r in rows if num(r[2]) is not None]
-        power = [num(r[3]) for r in rows if num(r[3]) is not None]
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "power_w_max": max(power) if power else None,
-                "samples": len(rows), "reasons": reasons}
+                self._proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self._proc.kill()
+            names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+            with open(self._path) as f:
+                for line in f:
+                    r = [x.strip() for x in line.split(",")]
+                    if len(r) < 9:
+                        continue
+                    try:
+                        self.samples.append((float(r[1]), float(r[3]),
+                                             [names[i] for i in range(4) if r[5 + i] == "Active"]))
+                        self.max_mhz = float(r[2])
+                    except ValueError:
+                        pass
+            os.unlink(self._path)
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no samples"],
+                    "source": self.source}
+        return {"sm_mhz": statistics.median(s[0] for s in self.samples),
+                "sm_max_mhz": self.max_mhz,
+                "sm_mhz_min": min(s[0] for s in self.samples),
+                "power_w_max": round(max(s[1] for s in self.samples), 1),
+                "power_limit_w": self.power_limit_w,
+                "samples": len(self.samples),
+                "reasons": sorted({r for s in self.samples for r in s[2]}),
+                "source": self.source}
 
 
 # ------------------------------------------------------------------------------ work model
@@ -195,9 +247,10 @@ def oracle_tokens_per_s(w, x_dev, wt, b, n_tokens, seed, cache=None):
 
 
 def default_sample(w):
-    # ~10-30 s of fp64 work on a few dozen host cores: scale by the per-token FFN work.
+    # ~10-30 s of fp64 work on a 16-core host (the full-size layer costs ~56 ms per token
+    # there): scale by the per-token FFN work.
     per_token = 6.0 * w.d * w.I * min(w.K, 9)
-    return int(max(4, min(w.T, 64, round(1.5e11 / per_token))))
+    return int(max(4, min(w.T, 512, round(2.0e11 / per_token))))
 
 
 # ------------------------------------------------------------------------------ our arm
@@ -208,12 +261,13 @@ def run_ours(args, rank, world, local_rank):
     log(f"[rank {rank}] generating {w.name} weights ({w.weight_bytes / 1e9:.1f} GB)")
     wt = make_weights(w, device, seed=args.seed)
     x = make_tokens(w, device, seed=args.seed + rank)
-    dm = mb.dims(w.T, w.d, w.N, w.Z, w.K, w.I)
+    dm = mb.dims(w.T, w.d, w.N, w.Z, w.K, w.I,
+                 flags=mb.RENORMALIZE_GATES if args.renormalize_gates else 0)
     ws = mb.alloc_workspace(dm, device)
     y = torch.empty((w.T, w.d), dtype=torch.bfloat16, device=device)
     b = wt["b"].clone()
     pid_state = torch.zeros(2, dtype=torch.float32, device=device)
-    params = mb.PidParams(w.pid_target, *PID_GAINS)
+    params = mb.PidParams(w.pid_target, *PID_GAINS, args.balance_gamma)
     n_steps = args.warmup + args.steps
     counts = torch.zeros((n_steps + args.steps, w.E), dtype=torch.int32, device=device)
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(mb.NUM_STAGE_EVENTS)]
@@ -265,11 +319,13 @@ def run_ours(args, rank, world, local_rank):
     tot_flops = {k: 0 for k in ("router_gemm", "ffn_up_gemm", "ffn_down_gemm")}
     tot_bytes = {k: 0 for k in ("router_gemm", "ffn_up_gemm", "ffn_down_gemm", "dispatch",
                                 "combine")}
-    A_steps, U_steps = [], []
+    A_steps, U_steps, load_ratio = [], [], []
     for c in hist:
         A, U, fl, by = work_model(w, c)
         A_steps.append(A)
         U_steps.append(U)
+        ffn = c[:w.N]
+        load_ratio.append(float(ffn.max()) / max(float(ffn.mean()), 1e-30))
         for k in fl:
             tot_flops[k] += fl[k]
         for k in by:
@@ -290,50 +346,92 @@ def run_ours(args, rank, world, local_rank):
                 "unit": "TFLOP/s"}
         peak_name = "bf16_tflops_sustained"
     roof["frac"] = round(achieved / peak, 4)
+    # the datasheet figures (dense bf16 2250 TFLOP/s, HBM3e 8000 GB/s), for context
+    roof["frac_of_nominal"] = round(achieved / (NOMINAL_HBM_GBS if roof["bound"] == "hbm"
+                                                else NOMINAL_BF16_TFLOPS), 4)
     tr = NCU_TRAFFIC.get((w.name, kernel))
     roof["traffic"] = tr["bytes_per_launch"] if tr and tr["src"] == gemm_source_hash() else None
     roof["kernel"] = kernel
     roof["peak_source"] = f"{pk_src} {peak_name}"
     layer_flops = sum(tot_flops.values())
-    layer = {"tflops": round(layer_flops / (ms / 1e3) / 1e12, 1),
-             "frac_of_bf16_peak": round(layer_flops / (ms / 1e3) / 1e12 / pk["bf16_tflops"], 4)}
+    layer_tflops = layer_flops / (ms / 1e3) / 1e12
+    layer_gbs = sum(tot_bytes.values()) / (ms / 1e3) / 1e9
+    routing = (A_steps, U_steps, load_ratio)
+    layer = {"tflops": round(layer_tflops, 1),
+             "frac_of_bf16_peak": round(layer_tflops / pk["bf16_tflops"], 4),
+             "frac_of_nominal_bf16": round(layer_tflops / NOMINAL_BF16_TFLOPS, 4),
+             "gbs": round(layer_gbs, 1),
+             "frac_of_hbm_peak": round(layer_gbs / pk["hbm_gbs"], 4),
+             "frac_of_nominal_hbm": round(layer_gbs / NOMINAL_HBM_GBS, 4)}
 
     # ---------------------------------------------------------------- end to end, host buffers
     if args.no_e2e:
-        return finish(args, w, world, rank, ms_max, A_steps, U_steps, roof, layer, stage_ms,
+        return finish(args, w, world, rank, ms_max, routing, roof, layer, stage_ms,
                       clk, None, x, wt, b)
+    # Pipelined like a serving loop: step i+1's input is copied host -> device on one copy
+    # stream and step i-1's output device -> host on another while step i computes; every
+    # step still moves its full input and output across the bus inside the timed region.
     x_host = torch.empty((w.T, w.d), dtype=torch.bfloat16).pin_memory()
     x_host.copy_(x.cpu())
-    y_host = torch.empty((w.T, w.d), dtype=torch.bfloat16).pin_memory()
-    x_dev = torch.empty_like(x)
+    y_host = [torch.empty((w.T, w.d), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    x_dev = [torch.empty_like(x) for _ in range(2)]
+    y_dev = [torch.empty_like(y) for _ in range(2)]
+    cs = torch.cuda.current_stream()
+    hs, ds = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
     e2e_steps = args.steps
-    for i in range(2):  # warm the copy path
-        x_dev.copy_(x_host, non_blocking=True)
-        step(n_steps + i)
-        y_host.copy_(y, non_blocking=True)
+
+    def e2e_run(n):
+        h2d_done, comp_done, d2h_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+        hs.wait_stream(cs)
+        ds.wait_stream(cs)
+        with torch.cuda.stream(hs):
+            x_dev[0].copy_(x_host, non_blocking=True)
+            h2d_done[0].record(hs)
+        for i in range(n):
+            cur = i % 2
+            if i + 1 < n:
+                nxt = (i + 1) % 2
+                if i >= 1:
+                    hs.wait_event(comp_done[nxt])  # step i-1 has finished reading x_dev[nxt]
+                with torch.cuda.stream(hs):
+                    x_dev[nxt].copy_(x_host, non_blocking=True)
+                    h2d_done[nxt].record(hs)
+            cs.wait_event(h2d_done[cur])
+            if i >= 2:
+                cs.wait_event(d2h_done[cur])  # y_dev[cur] of step i-2 has left the device
+            c = counts[n_steps + (i % args.steps)]
+            mb.moe_forward(dm, x_dev[cur], wt["W_r"], b, wt["W_g"], wt["W_u"], wt["W_d"],
+                           y_dev[cur], c, ws, stream=cs)
+            mb.moe_bias_update(dm, c, b, pid_state, params, stream=cs)
+            comp_done[cur].record(cs)
+            ds.wait_event(comp_done[cur])
+            with torch.cuda.stream(ds):
+                y_host[cur].copy_(y_dev[cur], non_blocking=True)
+                d2h_done[cur].record(ds)
+        cs.wait_stream(ds)
+        cs.wait_stream(hs)
+
+    e2e_run(2)  # warm the copy path
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(e2e_steps):
-        x_dev.copy_(x_host, non_blocking=True)
-        mb.moe_forward(dm, x_dev, wt["W_r"], b, wt["W_g"], wt["W_u"], wt["W_d"], y,
-                       counts[n_steps + (i % args.steps)], ws)
-        mb.moe_bias_update(dm, counts[n_steps + (i % args.steps)], b, pid_state, params)
-        y_host.copy_(y, non_blocking=True)
-    e1.record(stream)
+    e0.record(cs)
+    e2e_run(e2e_steps)
+    e1.record(cs)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
     e2e = {"value": round(job_throughput(world, w.T, e2e_steps, e2e_ms), 1), "unit": UNIT,
            "h2d_bytes_per_step": int(x_host.numel() * 2),
-           "d2h_bytes_per_step": int(y_host.numel() * 2)}
-    return finish(args, w, world, rank, ms_max, A_steps, U_steps, roof, layer, stage_ms, clk,
+           "d2h_bytes_per_step": int(y_host[0].numel() * 2),
+           "pipelined": "input and output copies on two copy streams, overlapped with compute"}
+    return finish(args, w, world, rank, ms_max, routing, roof, layer, stage_ms, clk,
                   e2e, x, wt, b)
 
 
-def finish(args, w, world, rank, ms_max, A_steps, U_steps, roof, layer, stage_ms, clk, e2e,
-           x, wt, b):
+def finish(args, w, world, rank, ms_max, routing, roof, layer, stage_ms, clk, e2e, x, wt, b):
+    A_steps, U_steps, load_ratio = routing
     result = {
         "metric": METRIC, "value": round(job_throughput(world, w.T, args.steps, ms_max), 1),
         "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -347,8 +445,11 @@ def finish(args, w, world, rank, ms_max, A_steps, U_steps, roof, layer, stage_ms
                   % (w.weight_bytes / 1e9, w.T * w.d * 2 / 1e6),
             "step": "moe_forward + moe_bias_update (PID target %.1f, kp=%g ki=%g kd=%g)"
                     % ((w.pid_target,) + PID_GAINS),
+            "variant": {"renormalize_gates": bool(args.renormalize_gates),
+                        "balance_gamma": args.balance_gamma},
             "mean_ffn_experts_per_token": round(float(np.mean(A_steps)) / w.T, 4),
             "distinct_ffn_experts": int(np.mean(U_steps)),
+            "ffn_load_max_over_mean": round(float(np.mean(load_ratio)), 2),
         },
         "roofline": roof,
         "layer": layer,
@@ -421,6 +522,10 @@ def main():
     ap.add_argument("--cpu-sample", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg (profiling)")
+    ap.add_argument("--renormalize-gates", action="store_true",
+                    help="variant: gates renormalised over the K selected experts")
+    ap.add_argument("--balance-gamma", type=float, default=0.0,
+                    help="variant: step of the per-expert balancing term after the PID step")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -21,7 +21,8 @@
  *     contiguous.  Shapes use the dims struct: T tokens, d model width, N FFN experts of
  *     intermediate width I, Z zero experts, K experts per token.
  *   - Limits: T >= 0; d and I positive multiples of 64; N >= 0, Z >= 0, 1 <= N + Z <= 1024;
- *     1 <= K <= min(N + Z, 32); T * K < 2^31.  Violations return MOE_ERR_SHAPE.
+ *     1 <= K <= min(N + Z, 32); T * K < 2^31; flags a combination of the MOE_* flags below.
+ *     Violations return MOE_ERR_SHAPE.
  *   - Every tensor pointer must be 16-byte aligned (MOE_ERR_ALIGN otherwise); a workspace
  *     must be 256-byte aligned.  A NULL required pointer returns MOE_ERR_ARG.
  *   - Errors are reported by the return code before anything is enqueued; a launch failure
@@ -52,14 +53,22 @@ typedef struct {
     int32_t Z; /* zero-computation experts (ids N .. N+Z-1) */
     int32_t K; /* experts selected per token */
     int32_t I; /* intermediate width of each SwiGLU FFN expert */
+    uint32_t flags; /* variant switches (MOE_RENORMALIZE_GATES); 0 = the layer as defined */
 } moe_dims;
 
-/* PID gains and set-point: target = desired mean number of FFN experts per token. */
+/* Gates renormalised over the selected set: g_i = p_i / sum of p over the K selected experts
+ * (zero experts included), instead of the layer's unrenormalised p_i.  An optional variant;
+ * it changes moe_route's topk_gate and hence everything downstream, not the selection. */
+#define MOE_RENORMALIZE_GATES 1u
+
+/* PID gains and set-point: target = desired mean number of FFN experts per token.
+ * balance_gamma: step of the per-expert balancing term (see moe_bias_update); 0 = off. */
 typedef struct {
     float target;
     float kp;
     float ki;
     float kd;
+    float balance_gamma;
 } moe_pid_params;
 
 enum {
@@ -101,7 +110,8 @@ size_t moe_scratch_size(const moe_dims *dims);
  *                                   tensor cores)
  *   b        [N+Z] fp32             per-expert selection bias
  *   topk_idx [T, K] int32   (out)   selected expert ids, ascending
- *   topk_gate[T, K] fp32    (out)   g_i = softmax(l)_i of the selected ids (not renormalised)
+ *   topk_gate[T, K] fp32    (out)   g_i = softmax(l)_i of the selected ids (not renormalised;
+ *                                   with MOE_RENORMALIZE_GATES divided by their fp32 sum)
  *   gap      [T] fp32       (out, nullable)  s_(K) - s_(K+1) with s = softmax(l) + b
  *                                   (+inf when K == N+Z); a small gap marks a near-tie
  * Exact score ties go to the lower expert id. */
@@ -169,6 +179,11 @@ int moe_combine(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *y_perm,
  *   m = sum_{i<N} counts[i] / T;  e = (target - m) / K;  integral += e;
  *   u = kp*e + ki*integral + kd*(e - e_prev);  e_prev = e;  b[i] += u for i < N.
  * fp32, one rounding per operation in that order (bit-reproducible on the host).
+ * Then, when params->balance_gamma != 0, the per-expert term of the aux-loss-free bias scheme
+ * that the PID refines (same section: the expert-specific bias follows recent expert usage;
+ * the rule is that scheme's published one): b[i] += balance_gamma * sign(mean - counts[i]) for
+ * i < N, mean = sum_{i<N} counts[i] / N, the sign taken exactly from the integers
+ * (sign(total - N*counts[i])).  balance_gamma must be finite (MOE_ERR_ARG otherwise).
  *   counts    [N+Z] int32 (as written by moe_dispatch / moe_forward)
  *   b         [N+Z] fp32  (in/out)  zero-expert biases are not changed
  *   pid_state [2] fp32    (in/out)  {integral, e_prev}; zero-initialise before the first step

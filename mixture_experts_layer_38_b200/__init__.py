@@ -3,12 +3,13 @@
 The work happens in libmoe_b200.so (C ABI: include/moe.h); this package is its thin binding
 (:mod:`.binding`) plus the seeded synthetic workloads (:mod:`.workloads`).
 """
-from .binding import (Dims, MoeError, PidParams, alloc_workspace, dims, moe_bias_update,
+from .binding import (RENORMALIZE_GATES, Dims, MoeError, PidParams, alloc_workspace, dims,
+                      moe_bias_update,
                       moe_combine, moe_dispatch, moe_expert_ffn, moe_forward,
                       moe_last_device_error, moe_route, scratch_size, strerror, workspace_size)
 
 __all__ = [
-    "Dims", "MoeError", "PidParams", "alloc_workspace", "dims", "moe_bias_update", "moe_combine",
+    "RENORMALIZE_GATES", "Dims", "MoeError", "PidParams", "alloc_workspace", "dims", "moe_bias_update", "moe_combine",
     "moe_dispatch", "moe_expert_ffn", "moe_forward", "moe_last_device_error", "moe_route",
     "scratch_size", "strerror", "workspace_size",
 ]

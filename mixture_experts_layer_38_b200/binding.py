@@ -36,15 +36,17 @@ class MoeError(RuntimeError):
 
 class Dims(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("N", ctypes.c_int32),
-                ("Z", ctypes.c_int32), ("K", ctypes.c_int32), ("I", ctypes.c_int32)]
+                ("Z", ctypes.c_int32), ("K", ctypes.c_int32), ("I", ctypes.c_int32),
+                ("flags", ctypes.c_uint32)]
 
     def __repr__(self):
-        return f"Dims(T={self.T}, d={self.d}, N={self.N}, Z={self.Z}, K={self.K}, I={self.I})"
+        return (f"Dims(T={self.T}, d={self.d}, N={self.N}, Z={self.Z}, K={self.K}, I={self.I}, "
+                f"flags={self.flags})")
 
 
 class PidParams(ctypes.Structure):
     _fields_ = [("target", ctypes.c_float), ("kp", ctypes.c_float), ("ki", ctypes.c_float),
-                ("kd", ctypes.c_float)]
+                ("kd", ctypes.c_float), ("balance_gamma", ctypes.c_float)]
 
 
 _lib = None
@@ -86,8 +88,11 @@ def lib():
     return _lib
 
 
-def dims(T, d, N, Z, K, I) -> Dims:
-    return Dims(int(T), int(d), int(N), int(Z), int(K), int(I))
+RENORMALIZE_GATES = 1  # MOE_RENORMALIZE_GATES
+
+
+def dims(T, d, N, Z, K, I, flags=0) -> Dims:
+    return Dims(int(T), int(d), int(N), int(Z), int(K), int(I), int(flags))
 
 
 def strerror(code: int) -> str:

@@ -9,7 +9,8 @@
 //   expert id, then the zero term, one bf16 rounding.
 // Same section, last paragraph: a PID controller tunes the expert biases from recent expert
 //   usage so the activated amount per token holds near a target (law: see moe_bias_update in
-//   the public header).
+//   the public header).  Optionally followed by the per-expert term of the aux-loss-free
+//   scheme the PID refines: b_i += gamma * sign(mean load - load_i), sign from integers.
 #include "device.cuh"
 #include "kernels.cuh"
 
@@ -77,7 +78,7 @@ __global__ void __launch_bounds__(kCombineThreads)
 
 __global__ void __launch_bounds__(256)
     pid_kernel(const int32_t *__restrict__ counts, int N, int K, int T, float *b, float *state,
-               float target, float kp, float ki, float kd) {
+               float target, float kp, float ki, float kd, float gamma) {
   __shared__ long long part[256];
   __shared__ float s_u;
   long long sum = 0;
@@ -102,7 +103,15 @@ __global__ void __launch_bounds__(256)
   }
   __syncthreads();
   const float u = s_u;
-  for (int i = threadIdx.x; i < N; i += blockDim.x) b[i] = __fadd_rn(b[i], u);
+  const long long total = part[0];
+  for (int i = threadIdx.x; i < N; i += blockDim.x) {
+    float bi = __fadd_rn(b[i], u);
+    if (gamma != 0.f) {
+      const long long diff = total - (long long)N * counts[i];
+      bi = __fadd_rn(bi, diff > 0 ? gamma : (diff < 0 ? -gamma : 0.f));
+    }
+    b[i] = bi;
+  }
 }
 
 }  // namespace
@@ -118,9 +127,10 @@ cudaError_t launch_combine(const uint16_t *x, const uint16_t *y_perm, const int3
 }
 
 cudaError_t launch_pid(const int32_t *counts, int N, int K, int T, float *b, float *state,
-                       float target, float kp, float ki, float kd, cudaStream_t stream) {
+                       float target, float kp, float ki, float kd, float gamma,
+                       cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
-  pid_kernel<<<1, 256, 0, stream>>>(counts, N, K, T, b, state, target, kp, ki, kd);
+  pid_kernel<<<1, 256, 0, stream>>>(counts, N, K, T, b, state, target, kp, ki, kd, gamma);
   return cudaGetLastError();
 }
 

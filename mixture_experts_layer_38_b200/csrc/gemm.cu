@@ -9,18 +9,21 @@
 //
 // Orientation: the pages' serving stack puts the weights on the MMA's M side and the tokens on
 // N ("SwapAB"), because N may be small and irregular.  The same holds for tcgen05: with M = 128,
-// N may be any multiple of 16 up to 256, so a tile is 2 x (128 weight rows) x (n <= 128
-// tokens): two accumulators share one token tile.  For the up-projection the two weight
+// N may be any multiple of 16 up to 256, so a tile is 2 x (128 weight rows) x (n <= 128 or 256
+// tokens, see Cfg): two accumulators share one token tile.  For the up-projection the two weight
 // sub-tiles are 128 rows of W_g and the same 128 rows of W_u, so each TMEM lane (thread) holds
 // the gate and the up value of one feature and SwiGLU needs no data exchange.  For the down
 // projection and the router they are 256 consecutive output rows.
 //
-// Warp roles (192 threads, one CTA per SM, persistent over a static tile schedule):
+// Warp roles (64 + 32 x kGemmEpiWarps = 192 threads, one CTA per SM, persistent over a static
+// tile schedule):
 //   warp 0      TMA producer: A0/A1 weight tiles (128 x 64) and the token tile (n x 64, issued
-//               as 128/64/32/16-row boxes) into a 4-stage ring of 48 KB stages
-//   warp 1      TMEM allocator (512 columns = 2 buffers x 2 accumulators x 128) and MMA issuer
+//               as 256/128/64/32/16-row boxes) into a 192 KB ring of 48 KB or 64 KB stages
+//   warp 1      TMEM allocator (512 columns: 2 buffers x 2 x 128, or 1 x 2 x 256) and MMA issuer
 //   warps 2-5   epilogue: tcgen05.ld from TMEM, fused SwiGLU / gate scaling / fp32 store via a
-//               per-warp shared-memory transpose and coalesced row stores
+//               per-warp shared-memory transpose and coalesced row stores.  A warp may only
+//               read the TMEM lane quarter (warp id mod 4); with more than four epilogue warps
+//               the warps of a quarter take alternate 32-token chunks of the tile.
 // Token tiles come in two kinds: full 128-row tiles (compute-bound) and each expert's partial
 // tail tile (for the many lightly loaded experts: weight streaming).  The static schedule
 // interleaves the two lists in proportion, and within a token tile the weight tiles come
@@ -37,22 +40,36 @@ namespace {
 
 constexpr int kBK = 64;                      // reduction elements per stage (128-byte rows)
 constexpr int kBM = 128;                     // weight rows per MMA
-constexpr int kBN = 128;                     // max token rows per tile
-constexpr int kStages = 4;
-constexpr int kTileA = kBM * kBK * 2;        // 16 KB
-constexpr int kTileB = kBN * kBK * 2;        // 16 KB
-constexpr int kStageBytes = 2 * kTileA + kTileB;
-constexpr int kEpiWarps = 4;
-constexpr int kStagingFloats = 32 * 32;      // per epilogue warp
+constexpr int kTileA = kBM * kBK * 2;        // 16 KB per weight block
+// Adjacent 128-row weight blocks and full 256-token tiles are fetched as single 256-row boxes
+// (fewer TMA operations for the one producer thread to issue).
+constexpr bool kWideBoxes = true;
+constexpr int kEpiWarps = kGemmEpiWarps;
+constexpr int kEpiGroups = kEpiWarps / 4;    // warps sharing one TMEM lane quarter
+constexpr int kStagingFloats = 16 * 32;      // 2 KB per epilogue warp: 32 x 32 bf16 or 16 x 32 fp32
+static_assert(kEpiWarps % 4 == 0, "epilogue warps come in groups of four lane quarters");
 constexpr int kMaxGroups = 1024;
 constexpr int kTmemCols = 512;
 constexpr long long kDrainLimitCycles = 1ll << 30;
-
-constexpr int kSmemStages = kStages * kStageBytes;
 constexpr int kSmemStaging = kEpiWarps * kStagingFloats * 4;
 constexpr int kSmemPrefix = 2 * (kMaxGroups + 4) * 4;  // full-tile and tail-tile prefixes
-constexpr int kNumBars = 2 * kStages + 4 + 1;
-constexpr int kSmemBytes = 1024 + kSmemStages + kSmemStaging + kSmemPrefix + kNumBars * 8 + 16;
+
+// Two tile widths.  BN = 128 tokens: 48 KB stages, 4 in a 192 KB ring (128 KB of weights in
+// flight, which weight-streaming tiles need), TMEM double-buffered (2 x 2 x 128 columns) so the
+// epilogue overlaps the next tile.  BN = 256: 64 KB stages, 3 in the ring, one 2 x 256-column
+// accumulator; every MMA and token load does twice the work, which is what compute-bound
+// tiles need (the issuing threads, not the tensor cores, limit 128-wide tiles).
+template <int BN>
+struct Cfg {
+  static constexpr int kAccBufs = BN <= 128 ? 2 : 1;
+  static constexpr int kStage = 2 * kTileA + BN * kBK * 2;
+  static constexpr int kStages = (192 * 1024) / kStage;
+  static constexpr int kNumBars = 2 * kStages + 2 * kAccBufs + 1;
+  static constexpr int kSmemBytes =
+      1024 + kStages * kStage + kSmemStaging + kSmemPrefix + kNumBars * 8 + 16;
+  static_assert(kAccBufs * 2 * BN <= kTmemCols, "TMEM holds 512 columns");
+  static_assert(kSmemBytes <= 232448, "shared memory per block");
+};
 
 struct Tile {
   int row0;     // first activation row
@@ -62,6 +79,7 @@ struct Tile {
   int a1_row;   // first weight row of sub-tile 1 in map_a1
   int m0;       // first output feature of the tile
   bool has_a1;  // sub-tile 1 exists
+  bool once;    // the group's only token tile: its weight tiles are read exactly once
   int kb0, kb1; // reduction blocks [kb0, kb1)
   int split;
 };
@@ -96,7 +114,7 @@ __device__ __forceinline__ int find_group(const int *pre, int G, int v) {
   return lo;
 }
 
-template <int EPI>
+template <int EPI, int BN>
 __device__ __forceinline__ Tile decode_tile(const GemmArgs &a, const Schedule &s, int tile) {
   Tile t;
   const int mt = tile % s.m_tiles;
@@ -110,13 +128,15 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs &a, const Schedule &s
   if (light_upto > light_before) {  // the (light_upto-1)-th tail tile
     g = find_group(s.lpre, s.G, light_upto - 1);
     const int lo = group_off(a, g), hi = group_off(a, g + 1);
-    t.row0 = lo + ((hi - lo) / kBN) * kBN;
+    t.row0 = lo + ((hi - lo) / BN) * BN;
     t.n_valid = hi - t.row0;
+    t.once = (hi - lo) < BN;
   } else {  // the (pos - light_before)-th full tile
     const int i = pos - light_before;
     g = find_group(s.hpre, s.G, i);
-    t.row0 = group_off(a, g) + (i - s.hpre[g]) * kBN;
-    t.n_valid = kBN;
+    t.row0 = group_off(a, g) + (i - s.hpre[g]) * BN;
+    t.n_valid = BN;
+    t.once = false;
   }
   t.nb = (t.n_valid + 15) & ~15;
   if (EPI == kEpiSwiGLU) {
@@ -160,6 +180,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *scratch, int &to
 
 // Full-tile and tail-tile prefixes over groups, computed by all threads of the block.  Returns
 // false (and records MOE_DEV_BAD_ROWS) if the offsets are not monotone or exceed the rows.
+template <int BN>
 __device__ bool build_schedule(const GemmArgs &a, int *hpre, int *lpre, int *scratch,
                                Schedule &s) {
   const int G = a.group_offsets ? a.num_groups : 1;
@@ -171,8 +192,8 @@ __device__ bool build_schedule(const GemmArgs &a, int *hpre, int *lpre, int *scr
   for (int g = g_begin; g < g_end; ++g) {
     const int lo = group_off(a, g), hi = group_off(a, g + 1);
     if (lo < 0 || hi < lo || hi > a.rows) { bad = true; continue; }
-    nh += (hi - lo) / kBN;
-    nl += ((hi - lo) % kBN) != 0;
+    nh += (hi - lo) / BN;
+    nl += ((hi - lo) % BN) != 0;
   }
   int H = 0, L = 0;
   int hrun = block_exclusive_scan(nh, scratch, H);
@@ -182,8 +203,8 @@ __device__ bool build_schedule(const GemmArgs &a, int *hpre, int *lpre, int *scr
     lpre[g] = lrun;
     const int lo = group_off(a, g), hi = group_off(a, g + 1);
     if (!(lo < 0 || hi < lo || hi > a.rows)) {
-      hrun += (hi - lo) / kBN;
-      lrun += ((hi - lo) % kBN) != 0;
+      hrun += (hi - lo) / BN;
+      lrun += ((hi - lo) % BN) != 0;
     }
   }
   if (threadIdx.x == 0) {
@@ -224,14 +245,14 @@ __device__ __forceinline__ float silu(float z) { return z / (1.0f + __expf(-z));
 // Thread `lane` of epilogue warp with TMEM lane quarter q owns output feature (q*32 + lane) of
 // each 128-row sub-tile; after the transpose through `stage` each thread stores 16 bytes of a
 // token row.
-template <int EPI>
+template <int EPI, int BN>
 __device__ __forceinline__ void epilogue_chunk(const GemmArgs &a, const Tile &t, uint32_t tcol,
                                                int chunk, int q, int lane, float *stage) {
   const int tok0 = chunk * 32;
   if (EPI == kEpiSwiGLU) {
     uint32_t g[32], u[32];
     tmem_ld_32x32b_x32(tcol, g);
-    tmem_ld_32x32b_x32(tcol + kBM, u);
+    tmem_ld_32x32b_x32(tcol + BN, u);
     tmem_ld_wait();
     uint16_t *st = reinterpret_cast<uint16_t *>(stage);
 #pragma unroll
@@ -262,7 +283,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs &a, const Tile &t,
     for (int sub = 0; sub < 2; ++sub) {
       if (sub == 1 && !t.has_a1) break;
       uint32_t v[32];
-      tmem_ld_32x32b_x32(tcol + sub * kBM, v);
+      tmem_ld_32x32b_x32(tcol + sub * BN, v);
       tmem_ld_wait();
       const int fbase = t.m0 + sub * kBM + q * 32;
       if (EPI == kEpiGated) {
@@ -285,55 +306,61 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs &a, const Tile &t,
           }
         }
         __syncwarp();
-      } else {  // kEpiF32
-#pragma unroll
-        for (int j = 0; j < 32; ++j) stage[j * 32 + lane] = __uint_as_float(v[j]);
-        __syncwarp();
+      } else {  // kEpiF32: two passes of 16 tokens through the staging buffer
         const int f = fbase + (lane & 7) * 4;
         float *out = reinterpret_cast<float *>(a.out) + (long long)t.split * a.split_stride;
 #pragma unroll
-        for (int it = 0; it < 8; ++it) {
-          const int r = it * 4 + (lane >> 3);
-          const int tok = tok0 + r;
-          if (tok < t.n_valid && f < a.M) {
-            const float4 val = *reinterpret_cast<const float4 *>(stage + r * 32 + (lane & 7) * 4);
-            *reinterpret_cast<float4 *>(out + (long long)(t.row0 + tok) * a.out_ld + f) = val;
+        for (int half = 0; half < 2; ++half) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) stage[j * 32 + lane] = __uint_as_float(v[half * 16 + j]);
+          __syncwarp();
+#pragma unroll
+          for (int it = 0; it < 4; ++it) {
+            const int r = it * 4 + (lane >> 3);
+            const int tok = tok0 + half * 16 + r;
+            if (tok < t.n_valid && f < a.M) {
+              const float4 val =
+                  *reinterpret_cast<const float4 *>(stage + r * 32 + (lane & 7) * 4);
+              *reinterpret_cast<float4 *>(out + (long long)(t.row0 + tok) * a.out_ld + f) = val;
+            }
           }
+          __syncwarp();
         }
-        __syncwarp();
       }
     }
   }
 }
 
-template <int EPI>
+template <int EPI, int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ GemmArgs args) {
+  using C = Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t *ring = smem;
-  float *staging = reinterpret_cast<float *>(smem + kSmemStages);
-  int *hpre = reinterpret_cast<int *>(smem + kSmemStages + kSmemStaging);
+  constexpr int kRing = C::kStages * C::kStage;
+  float *staging = reinterpret_cast<float *>(smem + kRing);
+  int *hpre = reinterpret_cast<int *>(smem + kRing + kSmemStaging);
   int *lpre = hpre + kMaxGroups + 4;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kSmemStages + kSmemStaging + kSmemPrefix);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kRing + kSmemStaging + kSmemPrefix);
   uint64_t *full_bar = bars;
-  uint64_t *empty_bar = bars + kStages;
-  uint64_t *tfull_bar = bars + 2 * kStages;
-  uint64_t *tempty_bar = bars + 2 * kStages + 2;
-  uint64_t *drain_bar = bars + 2 * kStages + 4;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kNumBars);
+  uint64_t *empty_bar = bars + C::kStages;
+  uint64_t *tfull_bar = bars + 2 * C::kStages;
+  uint64_t *tempty_bar = bars + 2 * C::kStages + C::kAccBufs;
+  uint64_t *drain_bar = bars + 2 * C::kStages + 2 * C::kAccBufs;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::kNumBars);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < C::kAccBufs; ++b) {
       mbar_init(&tfull_bar[b], 1);
       mbar_init(&tempty_bar[b], kEpiWarps);
     }
@@ -344,6 +371,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&args.map_a0);
     tma_prefetch_desc(&args.map_a1);
+    tma_prefetch_desc(&args.map_a01);
+    tma_prefetch_desc(&args.map_b256);
 #pragma unroll
     for (int i = 0; i < 4; ++i) tma_prefetch_desc(&args.map_b[i]);
   }
@@ -352,7 +381,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tmem_relinquish();
   }
   Schedule sched;
-  build_schedule(args, hpre, lpre, reinterpret_cast<int *>(staging), sched);
+  build_schedule<BN>(args, hpre, lpre, reinterpret_cast<int *>(staging), sched);
   sched.m_tiles = m_tiles_of<EPI>(args.M);
   sched.splits = EPI == kEpiF32 ? args.k_splits : 1;
   sched.total = sched.total * sched.m_tiles * sched.splits;
@@ -364,32 +393,48 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
-      const uint64_t pol_w = l2_policy_evict_normal();
+      // Weights of a group with a single token tile are read once: stream them past L2
+      // (evict-first) so they do not push out the tiles other CTAs are still re-reading.
+      const uint64_t pol_w_reused = l2_policy_evict_normal();
+      const uint64_t pol_w_once = l2_policy_evict_first();
       const uint64_t pol_x = l2_policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
       long long issued = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < sched.total; tile += gridDim.x) {
-        const Tile t = decode_tile<EPI>(args, sched, tile);
+        const Tile t = decode_tile<EPI, BN>(args, sched, tile);
         const uint32_t bytes = kTileA * (t.has_a1 ? 2 : 1) + t.nb * kBK * 2;
+        const uint64_t pol_w = t.once ? pol_w_once : pol_w_reused;
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag)) {
             signal_abort(args, abort_flag);
             ok = false;
             break;
           }
-          uint8_t *sa0 = ring + stage * kStageBytes;
+          uint8_t *sa0 = ring + stage * C::kStage;
           uint8_t *sa1 = sa0 + kTileA;
           uint8_t *sb = sa0 + 2 * kTileA;
           const int kc = kb * kBK;
           mbar_arrive_expect_tx(&full_bar[stage], bytes);
-          tma_load_2d(sa0, &args.map_a0, &full_bar[stage], kc, t.a0_row, pol_w);
-          if (t.has_a1) tma_load_2d(sa1, &args.map_a1, &full_bar[stage], kc, t.a1_row, pol_w);
+          if (kWideBoxes && EPI != kEpiSwiGLU && t.has_a1) {
+            tma_load_2d(sa0, &args.map_a01, &full_bar[stage], kc, t.a0_row, pol_w);
+          } else {
+            tma_load_2d(sa0, &args.map_a0, &full_bar[stage], kc, t.a0_row, pol_w);
+            if (t.has_a1) tma_load_2d(sa1, &args.map_a1, &full_bar[stage], kc, t.a1_row, pol_w);
+          }
+          // Token rows in boxes of 256 / 128 (as many as needed), then 64 / 32 / 16.
           int r = 0;
+          if (kWideBoxes && t.nb == 256) {
+            tma_load_2d(sb, &args.map_b256, &full_bar[stage], kc, t.row0, pol_x);
+            r = 256;
+          }
+          for (; t.nb - r >= 128; r += 128)
+            tma_load_2d(sb + r * (kBK * 2), &args.map_b[0], &full_bar[stage], kc, t.row0 + r,
+                        pol_x);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int box = kBN >> i;
+          for (int i = 1; i < 4; ++i) {
+            const int box = 128 >> i;
             if (t.nb - r >= box) {
               tma_load_2d(sb + r * (kBK * 2), &args.map_b[i], &full_bar[stage], kc, t.row0 + r,
                           pol_x);
@@ -397,15 +442,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
           }
           ++issued;
-          if (++stage == kStages) { stage = 0; phase ^= 1; }
+          if (++stage == C::kStages) { stage = 0; phase ^= 1; }
         }
       }
       if (!ok) {
         // Drain the copies that may still be landing in the ring (bounded).
-        for (long long i = 1; i <= issued && i <= kStages; ++i) {
+        for (long long i = 1; i <= issued && i <= C::kStages; ++i) {
           const long long idx = issued - i;
-          const int s = (int)(idx % kStages);
-          const uint32_t par = (uint32_t)((idx / kStages) & 1);
+          const int s = (int)(idx % C::kStages);
+          const uint32_t par = (uint32_t)((idx / C::kStages) & 1);
           const long long t0 = clock64();
           while (!mbar_try_wait(&full_bar[s], par) && clock64() - t0 < kDrainLimitCycles) {}
         }
@@ -420,17 +465,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       bool any = false;
       for (int tile = blockIdx.x; ok && tile < sched.total; tile += gridDim.x, ++it) {
-        const Tile t = decode_tile<EPI>(args, sched, tile);
-        const int buf = it & 1;
-        const uint32_t use = (uint32_t)(it >> 1);
+        const Tile t = decode_tile<EPI, BN>(args, sched, tile);
+        const int buf = it % C::kAccBufs;
+        const uint32_t use = (uint32_t)(it / C::kAccBufs);
         if (!mbar_wait(&tempty_bar[buf], (use & 1) ^ 1, abort_flag)) {
           signal_abort(args, abort_flag);
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t d0 = tmem_base + buf * (2 * kBM);
-        const uint32_t d1 = d0 + kBM;
+        const uint32_t d0 = tmem_base + buf * (2 * BN);
+        const uint32_t d1 = d0 + BN;
         const uint32_t idesc = idesc_bf16_f32(kBM, t.nb);
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
           if (!mbar_wait(&full_bar[stage], phase, abort_flag)) {
@@ -439,7 +484,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t base = smem_u32(ring + stage * kStageBytes);
+          const uint32_t base = smem_u32(ring + stage * C::kStage);
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k) {
             const uint64_t bdesc = sw128_kmajor_desc(base + 2 * kTileA + k * 32);
@@ -449,7 +494,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           any = true;
           umma_commit(&empty_bar[stage]);
-          if (++stage == kStages) { stage = 0; phase ^= 1; }
+          if (++stage == C::kStages) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
         umma_commit(&tfull_bar[buf]);
@@ -462,21 +507,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // ---------------------------------------------------------------- epilogue warps
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int q = warp & 3;              // TMEM lane quarter this warp may access
+    const int group = (warp - 2) >> 2;   // the warps of a quarter take alternate 32-token chunks
     float *stage = staging + (warp - 2) * kStagingFloats;
     int it = 0;
     for (int tile = blockIdx.x; tile < sched.total; tile += gridDim.x, ++it) {
-      const Tile t = decode_tile<EPI>(args, sched, tile);
-      const int buf = it & 1;
-      const uint32_t use = (uint32_t)(it >> 1);
+      const Tile t = decode_tile<EPI, BN>(args, sched, tile);
+      const int buf = it % C::kAccBufs;
+      const uint32_t use = (uint32_t)(it / C::kAccBufs);
       if (!warp_wait(&tfull_bar[buf], use & 1, abort_flag)) {
         if (lane == 0) signal_abort(args, abort_flag);
         break;
       }
       tc_fence_after();
-      const uint32_t tcol = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * (2 * kBM);
+      const uint32_t tcol = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * (2 * BN);
       const int chunks = (t.n_valid + 31) / 32;
-      for (int c = 0; c < chunks; ++c) epilogue_chunk<EPI>(args, t, tcol + c * 32, c, q, lane, stage);
+      for (int c = group; c < chunks; c += kEpiGroups)
+        epilogue_chunk<EPI, BN>(args, t, tcol + c * 32, c, q, lane, stage);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty_bar[buf]);
@@ -491,36 +538,53 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
-}  // namespace
+template <int EPI, int BN>
+cudaError_t set_smem_limit() {
+  return cudaFuncSetAttribute(grouped_gemm_kernel<EPI, BN>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<BN>::kSmemBytes);
+}
 
-int gemm_smem_bytes() { return kSmemBytes; }
+template <int BN>
+cudaError_t launch_bn(int epi, const GemmArgs &args, int grid, cudaStream_t stream) {
+  constexpr int smem = Cfg<BN>::kSmemBytes;
+  switch (epi) {
+    case kEpiSwiGLU:
+      grouped_gemm_kernel<kEpiSwiGLU, BN><<<grid, kGemmThreads, smem, stream>>>(args);
+      break;
+    case kEpiGated:
+      grouped_gemm_kernel<kEpiGated, BN><<<grid, kGemmThreads, smem, stream>>>(args);
+      break;
+    default:
+      grouped_gemm_kernel<kEpiF32, BN><<<grid, kGemmThreads, smem, stream>>>(args);
+      break;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
 
 cudaError_t gemm_prepare(int device) {
   (void)device;
   cudaError_t e;
-  e = cudaFuncSetAttribute(grouped_gemm_kernel<kEpiSwiGLU>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(grouped_gemm_kernel<kEpiGated>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(grouped_gemm_kernel<kEpiF32>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if ((e = set_smem_limit<kEpiSwiGLU, 128>()) != cudaSuccess) return e;
+  if ((e = set_smem_limit<kEpiGated, 128>()) != cudaSuccess) return e;
+  if ((e = set_smem_limit<kEpiF32, 128>()) != cudaSuccess) return e;
+  if ((e = set_smem_limit<kEpiSwiGLU, 256>()) != cudaSuccess) return e;
+  if ((e = set_smem_limit<kEpiGated, 256>()) != cudaSuccess) return e;
+  return set_smem_limit<kEpiF32, 256>();
 }
 
-cudaError_t launch_grouped_gemm(int epi, const GemmArgs &args, int grid, cudaStream_t stream) {
-  switch (epi) {
-    case kEpiSwiGLU:
-      grouped_gemm_kernel<kEpiSwiGLU><<<grid, kGemmThreads, kSmemBytes, stream>>>(args);
-      break;
-    case kEpiGated:
-      grouped_gemm_kernel<kEpiGated><<<grid, kGemmThreads, kSmemBytes, stream>>>(args);
-      break;
-    default:
-      grouped_gemm_kernel<kEpiF32><<<grid, kGemmThreads, kSmemBytes, stream>>>(args);
-      break;
-  }
-  return cudaGetLastError();
+int gemm_tile_tokens(long long rows, int groups, int K) {
+  // 256-token tiles need enough rows per group to fill them (mean rows per group, an upper
+  // bound since zero-expert slots are counted too) and a long reduction, over which the
+  // single accumulator buffer's epilogue stall is amortised.  Otherwise 128.
+  return (rows >= 128ll * groups && K >= 4096) ? 256 : 128;
+}
+
+cudaError_t launch_grouped_gemm(int epi, const GemmArgs &args, int grid, int tile_tokens,
+                                cudaStream_t stream) {
+  return tile_tokens == 256 ? launch_bn<256>(epi, args, grid, stream)
+                            : launch_bn<128>(epi, args, grid, stream);
 }
 
 }  // namespace moe

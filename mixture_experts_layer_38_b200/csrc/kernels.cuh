@@ -9,7 +9,7 @@
 namespace moe {
 
 // ------------------------------------------------------------------ grouped GEMM (tcgen05)
-// Output tile = 2 x (128 weight rows) x (<= 128 activation rows); see gemm.cu.
+// Output tile = 2 x (128 weight rows) x (<= 128 or 256 activation rows); see gemm.cu.
 enum EpiKind : int {
   kEpiSwiGLU = 0,  // h = silu(A0 x) * (A1 x)           -> bf16 [rows, M]
   kEpiGated = 1,   // y = row_scale[r] * (A x)          -> bf16 [rows, M]
@@ -19,7 +19,10 @@ enum EpiKind : int {
 struct GemmArgs {
   CUtensorMap map_a0;    // weight rows (box 64 x 128)
   CUtensorMap map_a1;    // W_u for SwiGLU, the same tensor as map_a0 otherwise
+  CUtensorMap map_a01;   // map_a0's tensor in 64 x 256 boxes: both 128-row blocks at once when
+                         // they are adjacent rows (down projection, router)
   CUtensorMap map_b[4];  // activation rows, boxes of 128 / 64 / 32 / 16 rows x 64 columns
+  CUtensorMap map_b256;  // activation rows, boxes of 256 rows
   const int32_t *group_offsets;  // [num_groups + 1] activation-row offsets, or nullptr
   int num_groups;                // groups (experts); 1 when group_offsets == nullptr
   int rows;                      // activation rows available (bound for group_offsets)
@@ -33,16 +36,24 @@ struct GemmArgs {
   int *status;                   // device status word
 };
 
-constexpr int kGemmThreads = 192;
-int gemm_smem_bytes();
+// Grouped GEMM block: warp 0 issues TMA loads, warp 1 allocates TMEM and issues MMAs, and
+// kGemmEpiWarps warps (a multiple of 4: one per TMEM lane quarter, per group) drain TMEM.
+// Eight shortened the MMA thread's waits for a free accumulator at 256-token tiles but were no
+// faster: those tiles run at the board's power limit, where idle tensor cycles cost no time.
+constexpr int kGemmEpiWarps = 4;
+constexpr int kGemmThreads = 64 + 32 * kGemmEpiWarps;
 cudaError_t gemm_prepare(int device);  // sets the kernels' shared-memory limit once per device
-cudaError_t launch_grouped_gemm(int epi, const GemmArgs &args, int grid, cudaStream_t stream);
+// Token-tile width (128 or 256) for `rows` activation rows over `groups` groups, reduction K.
+int gemm_tile_tokens(long long rows, int groups, int K);
+cudaError_t launch_grouped_gemm(int epi, const GemmArgs &args, int grid, int tile_tokens,
+                                cudaStream_t stream);
 
 // ------------------------------------------------------------------ routing
 // logits [splits][T][E] fp32 -> softmax, biased top-K, ascending ids.
+// renormalize: gates divided by their sum over the K selected experts.
 cudaError_t launch_route_topk(const float *logits, int splits, int T, int E, int K,
-                              const float *b, int32_t *topk_idx, float *topk_gate, float *gap,
-                              int *status, cudaStream_t stream);
+                              const float *b, bool renormalize, int32_t *topk_idx,
+                              float *topk_gate, float *gap, int *status, cudaStream_t stream);
 
 // ------------------------------------------------------------------ dispatch
 constexpr int kDispatchChunk = 256;  // tokens per histogram chunk (8 warps x 32)
@@ -57,7 +68,9 @@ cudaError_t launch_dispatch(const uint16_t *x, const int32_t *topk_idx, const fl
 cudaError_t launch_combine(const uint16_t *x, const uint16_t *y_perm, const int32_t *topk_idx,
                            const float *topk_gate, const int32_t *slot_pos, int T, int d, int N,
                            int K, int rows, uint16_t *y, int *status, cudaStream_t stream);
+// PID step on the FFN biases, then (gamma != 0) the per-expert balancing term.
 cudaError_t launch_pid(const int32_t *counts, int N, int K, int T, float *b, float *state,
-                       float target, float kp, float ki, float kd, cudaStream_t stream);
+                       float target, float kp, float ki, float kd, float gamma,
+                       cudaStream_t stream);
 
 }  // namespace moe

@@ -3,6 +3,7 @@
 //
 // Every check happens on the host before anything is enqueued; nothing here synchronises
 // except moe_last_device_error, and nothing allocates device memory.
+#include <cmath>
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -88,7 +89,7 @@ bool make_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
 bool make_act_maps(GemmArgs &a, const void *base, uint64_t rows, uint64_t cols) {
   for (int i = 0; i < 4; ++i)
     if (!make_map(&a.map_b[i], base, rows, cols, 128u >> i)) return false;
-  return true;
+  return make_map(&a.map_b256, base, rows, cols, 256);
 }
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -102,6 +103,7 @@ bool dims_ok(const moe_dims *d) {
   if (d->K < 1 || d->K > kMaxK || d->K > E) return false;
   if ((long long)d->T * d->K >= (1ll << 31)) return false;
   if ((long long)d->N * d->I >= (1ll << 31) || (long long)d->N * d->d >= (1ll << 31)) return false;
+  if ((d->flags & ~MOE_RENORMALIZE_GATES) != 0) return false;
   return true;
 }
 
@@ -204,6 +206,7 @@ int do_route(const moe_dims &d, const DeviceInfo &di, const Layout &L, const moe
   GemmArgs a{};
   if (!make_map(&a.map_a0, W_r, (uint64_t)E, (uint64_t)d.d, 128) ||
       !make_map(&a.map_a1, W_r, (uint64_t)E, (uint64_t)d.d, 128) ||
+      !make_map(&a.map_a01, W_r, (uint64_t)E, (uint64_t)d.d, 256) ||
       !make_act_maps(a, x, (uint64_t)d.T, (uint64_t)d.d)) {
     return MOE_ERR_CUDA;
   }
@@ -220,11 +223,12 @@ int do_route(const moe_dims &d, const DeviceInfo &di, const Layout &L, const moe
   a.status = status;
   const long long tiles = (long long)((d.T + 127) / 128) * ((E + 255) / 256) * L.splits;
   const int grid = (int)(tiles < di.sms ? tiles : di.sms);
-  cudaError_t e = launch_grouped_gemm(kEpiF32, a, grid, stream);
+  cudaError_t e = launch_grouped_gemm(kEpiF32, a, grid, gemm_tile_tokens(d.T, 1, d.d), stream);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if (record(events, 1, stream) != MOE_OK) return MOE_ERR_CUDA;
   return to_status(
-      launch_route_topk(logits, L.splits, d.T, E, d.K, b, topk_idx, topk_gate, gap, status, stream));
+      launch_route_topk(logits, L.splits, d.T, E, d.K, b, (d.flags & MOE_RENORMALIZE_GATES) != 0,
+                        topk_idx, topk_gate, gap, status, stream));
 }
 
 int do_dispatch(const moe_dims &d, const DeviceInfo &di, const Layout &L, const moe_bf16 *x,
@@ -253,6 +257,7 @@ int do_expert_ffn(const moe_dims &d, const DeviceInfo &di, const Layout &L,
   GemmArgs up{};
   if (!make_map(&up.map_a0, W_g, (uint64_t)d.N * d.I, (uint64_t)d.d, 128) ||
       !make_map(&up.map_a1, W_u, (uint64_t)d.N * d.I, (uint64_t)d.d, 128) ||
+      !make_map(&up.map_a01, W_g, (uint64_t)d.N * d.I, (uint64_t)d.d, 256) ||
       !make_act_maps(up, x_perm, rows, (uint64_t)d.d)) {
     return MOE_ERR_CUDA;
   }
@@ -267,12 +272,15 @@ int do_expert_ffn(const moe_dims &d, const DeviceInfo &di, const Layout &L,
   up.split_stride = 0;
   up.row_scale = nullptr;
   up.status = status;
-  if (launch_grouped_gemm(kEpiSwiGLU, up, di.sms, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  const int tile_tokens = gemm_tile_tokens((long long)rows, d.N, d.d);
+  if (launch_grouped_gemm(kEpiSwiGLU, up, di.sms, tile_tokens, stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
   if (record(events, 4, stream) != MOE_OK) return MOE_ERR_CUDA;
 
   GemmArgs down{};
   if (!make_map(&down.map_a0, W_d, (uint64_t)d.N * d.d, (uint64_t)d.I, 128) ||
       !make_map(&down.map_a1, W_d, (uint64_t)d.N * d.d, (uint64_t)d.I, 128) ||
+      !make_map(&down.map_a01, W_d, (uint64_t)d.N * d.d, (uint64_t)d.I, 256) ||
       !make_act_maps(down, h, rows, (uint64_t)d.I)) {
     return MOE_ERR_CUDA;
   }
@@ -287,7 +295,7 @@ int do_expert_ffn(const moe_dims &d, const DeviceInfo &di, const Layout &L,
   down.split_stride = 0;
   down.row_scale = perm_gate;
   down.status = status;
-  return to_status(launch_grouped_gemm(kEpiGated, down, di.sms, stream));
+  return to_status(launch_grouped_gemm(kEpiGated, down, di.sms, tile_tokens, stream));
 }
 
 }  // namespace
@@ -417,11 +425,12 @@ int moe_bias_update(const moe_dims *dims, const int32_t *counts, float *b, float
   MOE_CHECK_PTR(counts);
   MOE_CHECK_PTR(b);
   MOE_CHECK_PTR(pid_state);
+  MOE_REQUIRE(std::isfinite(params->balance_gamma), MOE_ERR_ARG);
   const DeviceInfo *di = nullptr;
   const int rc = device_info(&di);
   if (rc != MOE_OK) return rc;
   return to_status(launch_pid(counts, dims->N, dims->K, dims->T, b, pid_state, params->target,
-                              params->kp, params->ki, params->kd,
+                              params->kp, params->ki, params->kd, params->balance_gamma,
                               static_cast<cudaStream_t>(stream)));
 }
 

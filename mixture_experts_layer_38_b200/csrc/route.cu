@@ -7,6 +7,7 @@
 //   p   = exp(l - max l) / sum exp(l - max l)
 //   s   = p + b;  the K largest s are selected, an exact tie going to the lower expert id
 //   out = selected ids in ascending order, gates g = p (not renormalised), gap = s_(K) - s_(K+1)
+//   (variant: g = p / sum of the K selected p, summed in a fixed shuffle order)
 // Thread i of the 256-thread block holds experts i, i+256, i+512, i+768 in registers, so the
 // split-K partial sums, exp and bias are spread over 8 warps; each of the K+1 selection rounds
 // is a block-wide argmax of one 64-bit key per thread, and the result does not depend on
@@ -56,8 +57,9 @@ __device__ __forceinline__ float block_reduce(float v, bool is_max, float *red) 
 
 __global__ void __launch_bounds__(kBlockThreads)
     route_topk_block_kernel(const float *__restrict__ logits, int splits, int T, int E, int ld,
-                            int K, const float *__restrict__ b, int32_t *__restrict__ topk_idx,
-                            float *__restrict__ topk_gate, float *__restrict__ gap, int *status) {
+                            int K, const float *__restrict__ b, bool renormalize,
+                            int32_t *__restrict__ topk_idx, float *__restrict__ topk_gate,
+                            float *__restrict__ gap, int *status) {
   __shared__ float red[kBlockThreads / 32];
   __shared__ uint64_t wbest[kBlockThreads / 32];
   __shared__ int sel_id[33];
@@ -113,6 +115,7 @@ __global__ void __launch_bounds__(kBlockThreads)
       if (tid == 0) {
         record_status(status, MOE_DEV_BAD_EXPERT);
         sel_id[k] = 0x7fffffff;
+        sel_p[k] = 0.f;
       }
     } else if (id % kBlockThreads == tid) {
       const int j = id / kBlockThreads;
@@ -136,9 +139,17 @@ __global__ void __launch_bounds__(kBlockThreads)
       const int other = __shfl_sync(0xffffffffu, my_id, k2);
       rank += other < my_id;
     }
+    float g = lane < K ? sel_p[lane] : 0.f;
+    if (renormalize) {
+      float sum = g;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1)
+        sum = __fadd_rn(sum, __shfl_xor_sync(0xffffffffu, sum, off));
+      g = __fdiv_rn(g, sum);
+    }
     if (lane < K) {
       topk_idx[(long long)t * K + rank] = my_id;
-      topk_gate[(long long)t * K + rank] = sel_p[lane];
+      topk_gate[(long long)t * K + rank] = g;
     }
     if (gap != nullptr && lane == 0)
       gap[t] = (K < E) ? __fsub_rn(sel_s[K - 1], sel_s[K]) : INFINITY;
@@ -148,12 +159,12 @@ __global__ void __launch_bounds__(kBlockThreads)
 }  // namespace
 
 cudaError_t launch_route_topk(const float *logits, int splits, int T, int E, int K,
-                              const float *b, int32_t *topk_idx, float *topk_gate, float *gap,
-                              int *status, cudaStream_t stream) {
+                              const float *b, bool renormalize, int32_t *topk_idx,
+                              float *topk_gate, float *gap, int *status, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
   const int ld = (E + 3) & ~3;
-  route_topk_block_kernel<<<T, kBlockThreads, 0, stream>>>(logits, splits, T, E, ld, K, b,
-                                                          topk_idx, topk_gate, gap, status);
+  route_topk_block_kernel<<<T, kBlockThreads, 0, stream>>>(
+      logits, splits, T, E, ld, K, b, renormalize, topk_idx, topk_gate, gap, status);
   return cudaGetLastError();
 }
 

@@ -91,9 +91,9 @@ def to_np(t):
 class Stages:
     """Device buffers for running the staged C-ABI calls on one workload."""
 
-    def __init__(self, w, x, wt, device="cuda"):
+    def __init__(self, w, x, wt, device="cuda", flags=0):
         self.w = w
-        self.dm = mb.dims(w.T, w.d, w.N, w.Z, w.K, w.I)
+        self.dm = mb.dims(w.T, w.d, w.N, w.Z, w.K, w.I, flags=flags)
         R = w.T * w.K
         i32 = dict(dtype=torch.int32, device=device)
         f32 = dict(dtype=torch.float32, device=device)

@@ -88,6 +88,19 @@ def test_argument_errors_are_reported_before_any_device_work():
     assert lib.moe_last_device_error(None, None) == 1
 
 
+def test_variant_switches_are_validated():
+    lib = mb.lib()
+    dm = mb.dims(64, 128, 8, 4, 3, 256, flags=mb.RENORMALIZE_GATES)
+    assert mb.workspace_size(dm) == mb.workspace_size(mb.dims(64, 128, 8, 4, 3, 256))
+    assert mb.workspace_size(mb.dims(64, 128, 8, 4, 3, 256, flags=2)) == 0  # unknown flag
+    assert _fwd(mb.dims(64, 128, 8, 4, 3, 256, flags=0x80)) == 2            # MOE_ERR_SHAPE
+    for gamma in (float("nan"), float("inf")):
+        params = mb.PidParams(8.0, 0.1, 0.0, 0.0, gamma)
+        assert lib.moe_bias_update(ctypes.byref(dm), P(0x10000), P(0x20000), P(0x30000),
+                                   ctypes.byref(params), None) == 1          # MOE_ERR_ARG
+    assert ctypes.sizeof(mb.Dims) == 28 and ctypes.sizeof(mb.PidParams) == 20
+
+
 def _replica_worker(rank, world, port, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
