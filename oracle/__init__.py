@@ -43,6 +43,14 @@ def _load():
         _lib.oracle_pid_step.argtypes = [_i64, _i64, _i64, _ptr, _ptr, _ptr, ctypes.c_float,
                                          ctypes.c_float, ctypes.c_float, ctypes.c_float]
         _lib.oracle_renormalize_gates.argtypes = [_i64, _i64, _ptr]
+        _lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        _lib.oracle_e4m3_decode.restype = ctypes.c_double
+        _lib.oracle_e4m3_encode.argtypes = [ctypes.c_double]
+        _lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+        _lib.oracle_quantize_fp8_blocks.argtypes = [_i64, _i64, _i64, _ptr, _ptr, _ptr]
+        _lib.oracle_quantize_fp8_blocks.restype = None
+        _lib.oracle_dequantize_fp8_blocks.argtypes = [_i64, _i64, _i64, _ptr, _ptr, _ptr]
+        _lib.oracle_dequantize_fp8_blocks.restype = None
         _lib.oracle_balance_step.argtypes = [_i64, _ptr, _ptr, ctypes.c_float]
         for f in ("oracle_router", "oracle_dispatch", "oracle_swiglu_expert",
                   "oracle_combine_tokens", "oracle_combine_rows", "oracle_forward",
@@ -249,3 +257,37 @@ def balance_step(counts, b, N, gamma):
     counts = _i32(counts)
     assert b.dtype == np.float32 and b.flags.c_contiguous
     _load().oracle_balance_step(N, _p(counts), _p(b), gamma)
+
+
+def e4m3_decode(code):
+    """Value of an E4M3 code (NaN for S.1111.111)."""
+    return float(_load().oracle_e4m3_decode(int(code)))
+
+
+def e4m3_encode(v):
+    """E4M3 code of v: nearest, ties to even mantissa, saturating at +-448."""
+    return int(_load().oracle_e4m3_encode(float(v)))
+
+
+def quantize_fp8_blocks(w):
+    """Block-wise FP8 of bf16 weights [G, R, C] (R, C multiples of 128): returns (q uint8
+    [G, R, C], scale float32 [G, R/128, C/128]), one power-of-two scale per 128 x 128 block."""
+    w = bf16_bits(w)
+    if w.ndim == 2:
+        w = w[None]
+    G, R, C = w.shape
+    assert R % 128 == 0 and C % 128 == 0
+    q = np.zeros((G, R, C), np.uint8)
+    scale = np.zeros((G, R // 128, C // 128), np.float32)
+    _load().oracle_quantize_fp8_blocks(G, R, C, _p(np.ascontiguousarray(w)), _p(q), _p(scale))
+    return q, scale
+
+
+def dequantize_fp8_blocks(q, scale):
+    """q * (its block's scale) as bf16 bit patterns [G, R, C] (the weights the FP8 variant uses)."""
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    scale = np.ascontiguousarray(scale, dtype=np.float32)
+    G, R, C = q.shape
+    w = np.zeros((G, R, C), np.uint16)
+    _load().oracle_dequantize_fp8_blocks(G, R, C, _p(q), _p(scale), _p(w))
+    return w

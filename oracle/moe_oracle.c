@@ -359,3 +359,97 @@ void oracle_balance_step(int64_t N, const int32_t *counts, float *b, float gamma
         b[i] = b[i] + gamma * s;
     }
 }
+
+/* ------------------------------------------------------------------------------------------
+ * FP8 block-quantised expert weights (an optional variant).  P1 §系統級優化 says LongCat-Flash
+ * quantises with the same fine-grained block-wise scheme as DeepSeek-V3, i.e. one scale per
+ * 128 x 128 block of a weight matrix.  Readings taken here (the page gives no format details): the element format is E4M3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits;
+ * no infinities; S.1111.111 is NaN; largest finite 448); each block's scale is the smallest
+ * power of two 2^e with max|w| <= 448 * 2^e (a power of two keeps q * 2^e exact in bf16);
+ * q = E4M3(w / 2^e) rounded to nearest, ties to even mantissa, saturating at +-448.
+ * Activations stay bf16 (weight-only quantisation).
+ * ---------------------------------------------------------------------------------------- */
+double oracle_e4m3_decode(uint8_t code)
+{
+    const int s = code >> 7, E = (code >> 3) & 15, M = code & 7;
+    if (E == 15 && M == 7) return NAN;
+    double v = (E == 0) ? ldexp((double)M, -9) : ldexp(1.0 + M / 8.0, E - 7);
+    return s ? -v : v;
+}
+
+uint8_t oracle_e4m3_encode(double v)
+{
+    if (isnan(v)) return 0x7F;
+    const uint8_t s = signbit(v) ? 0x80 : 0x00;
+    const double a = fabs(v);
+    if (a >= 448.0) return (uint8_t)(s | 0x7E);
+    if (a < ldexp(1.0, -6)) {                   /* subnormal grid: multiples of 2^-9 */
+        const double q = nearbyint(ldexp(a, 9)); /* ties to even under the default mode */
+        return (uint8_t)(s | (uint8_t)q);        /* q == 8 is the smallest normal, code 8 */
+    }
+    int x;
+    (void)frexp(a, &x);                          /* a = f * 2^x, f in [0.5, 1) */
+    int e = x - 1;                               /* a = m * 2^e, m in [1, 2) */
+    double mq = nearbyint((ldexp(a, -e) - 1.0) * 8.0);
+    if (mq == 8.0) { mq = 0.0; e += 1; }
+    return (uint8_t)(s | (uint8_t)(((e + 7) << 3) | (int)mq));
+}
+
+/* Round-to-nearest-even conversion of a double that is exact in fp32 to bf16 bits. */
+static uint16_t f64_to_bf16_rne(double v)
+{
+    float f = (float)v;
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7FFFFFFFu) > 0x7F800000u) return (uint16_t)((u >> 16) | 0x40); /* NaN */
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+
+/* w: G matrices of [R][C] bf16 (R, C multiples of 128) -> q [G][R][C] E4M3 codes and
+ * scale [G][R/128][C/128] fp32 (= 2^e). */
+void oracle_quantize_fp8_blocks(int64_t G, int64_t R, int64_t C, const uint16_t *w, uint8_t *q,
+                                float *scale)
+{
+    const int64_t RB = R / 128, CB = C / 128;
+#pragma omp parallel for schedule(static)
+    for (int64_t gb = 0; gb < G * RB; ++gb) {
+        const int64_t g = gb / RB, rb = gb % RB;
+        for (int64_t cb = 0; cb < CB; ++cb) {
+            double amax = 0.0;
+            for (int64_t r = 0; r < 128; ++r)
+                for (int64_t c = 0; c < 128; ++c) {
+                    const double a = fabs(bf16_to_f64(w[(g * R + rb * 128 + r) * C + cb * 128 + c]));
+                    if (a > amax) amax = a;
+                }
+            int e = 0;
+            if (amax > 0.0) {
+                e = ilogb(amax) - 8;
+                while (amax > ldexp(448.0, e)) ++e;
+                while (amax <= ldexp(448.0, e - 1)) --e;
+                if (e < -126) e = -126;
+            }
+            scale[(g * RB + rb) * CB + cb] = (float)ldexp(1.0, e);
+            for (int64_t r = 0; r < 128; ++r)
+                for (int64_t c = 0; c < 128; ++c) {
+                    const int64_t i = (g * R + rb * 128 + r) * C + cb * 128 + c;
+                    q[i] = oracle_e4m3_encode(ldexp(bf16_to_f64(w[i]), -e));
+                }
+        }
+    }
+}
+
+/* The weights the FP8 variant computes with: q * scale of its block, as bf16 bits (exact
+ * unless the product underflows bf16). */
+void oracle_dequantize_fp8_blocks(int64_t G, int64_t R, int64_t C, const uint8_t *q,
+                                  const float *scale, uint16_t *w)
+{
+    const int64_t RB = R / 128, CB = C / 128;
+    for (int64_t g = 0; g < G; ++g)
+        for (int64_t r = 0; r < R; ++r)
+            for (int64_t c = 0; c < C; ++c) {
+                const int64_t i = (g * R + r) * C + c;
+                const double s = (double)scale[(g * RB + r / 128) * CB + c / 128];
+                w[i] = f64_to_bf16_rne(oracle_e4m3_decode(q[i]) * s);
+            }
+}
