@@ -197,8 +197,10 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------ work model
-def work_model(w, counts):
-    """Algorithmic FLOPs and bytes of one step from the routing actually taken."""
+def work_model(w, counts, wb=2):
+    """Algorithmic FLOPs and bytes of one step from the routing actually taken; `wb` bytes per
+    expert weight (2 for bf16, 1 for the FP8 codes; their block scales add 4 bytes per 16384
+    weights, negligible)."""
     counts = np.asarray(counts, np.int64)
     A = int(counts[:w.N].sum())
     U = int((counts[:w.N] > 0).sum())
@@ -210,8 +212,8 @@ def work_model(w, counts):
     }
     bytes_ = {
         "router_gemm": E * d * 2 + T * d * 2 + T * E * 4,
-        "ffn_up_gemm": U * 2 * I * d * 2 + A * d * 2 + A * I * 2,
-        "ffn_down_gemm": U * d * I * 2 + A * I * 2 + A * d * 2,
+        "ffn_up_gemm": U * 2 * I * d * wb + A * d * 2 + A * I * 2,
+        "ffn_down_gemm": U * d * I * wb + A * I * 2 + A * d * 2,
         "dispatch": 2 * A * d * 2,
         "combine": (A + 2 * T) * d * 2,
     }
@@ -266,6 +268,21 @@ def run_ours(args, rank, world, local_rank):
     ws = mb.alloc_workspace(dm, device)
     y = torch.empty((w.T, w.d), dtype=torch.bfloat16, device=device)
     b = wt["b"].clone()
+    fw = None
+    if args.fp8:
+        log(f"[rank {rank}] quantising the expert weights to block-wise FP8")
+        fw = mb.quantize_expert_weights_fp8(dm, wt["W_g"], wt["W_u"], wt["W_d"])
+
+    def forward(x_in, y_out, c, ev=None, stream=None):
+        if fw is not None:
+            mb.moe_forward_fp8(dm, x_in, wt["W_r"], b, fw, y_out, c, ws, stream=stream,
+                               events=ev)
+        elif ev is None:
+            mb.moe_forward(dm, x_in, wt["W_r"], b, wt["W_g"], wt["W_u"], wt["W_d"], y_out, c, ws,
+                           stream=stream)
+        else:
+            mb.moe_forward_timed(dm, x_in, wt["W_r"], b, wt["W_g"], wt["W_u"], wt["W_d"], y_out,
+                                 c, ws, ev, stream=stream)
     pid_state = torch.zeros(2, dtype=torch.float32, device=device)
     params = mb.PidParams(w.pid_target, *PID_GAINS, args.balance_gamma)
     n_steps = args.warmup + args.steps
@@ -278,11 +295,7 @@ def run_ours(args, rank, world, local_rank):
             e.record(stream)
 
     def step(i, ev=None):
-        if ev is None:
-            mb.moe_forward(dm, x, wt["W_r"], b, wt["W_g"], wt["W_u"], wt["W_d"], y, counts[i], ws)
-        else:
-            mb.moe_forward_timed(dm, x, wt["W_r"], b, wt["W_g"], wt["W_u"], wt["W_d"], y,
-                                 counts[i], ws, ev)
+        forward(x, y, counts[i], ev)
         mb.moe_bias_update(dm, counts[i], b, pid_state, params)
 
     for i in range(args.warmup):
@@ -321,7 +334,7 @@ def run_ours(args, rank, world, local_rank):
                                 "combine")}
     A_steps, U_steps, load_ratio = [], [], []
     for c in hist:
-        A, U, fl, by = work_model(w, c)
+        A, U, fl, by = work_model(w, c, wb=1 if args.fp8 else 2)
         A_steps.append(A)
         U_steps.append(U)
         ffn = c[:w.N]
@@ -349,7 +362,7 @@ def run_ours(args, rank, world, local_rank):
     # the datasheet figures (dense bf16 2250 TFLOP/s, HBM3e 8000 GB/s), for context
     roof["frac_of_nominal"] = round(achieved / (NOMINAL_HBM_GBS if roof["bound"] == "hbm"
                                                 else NOMINAL_BF16_TFLOPS), 4)
-    tr = NCU_TRAFFIC.get((w.name, kernel))
+    tr = NCU_TRAFFIC.get((w.name + ("+fp8" if args.fp8 else ""), kernel))
     roof["traffic"] = tr["bytes_per_launch"] if tr and tr["src"] == gemm_source_hash() else None
     roof["kernel"] = kernel
     roof["peak_source"] = f"{pk_src} {peak_name}"
@@ -401,8 +414,7 @@ def run_ours(args, rank, world, local_rank):
             if i >= 2:
                 cs.wait_event(d2h_done[cur])  # y_dev[cur] of step i-2 has left the device
             c = counts[n_steps + (i % args.steps)]
-            mb.moe_forward(dm, x_dev[cur], wt["W_r"], b, wt["W_g"], wt["W_u"], wt["W_d"],
-                           y_dev[cur], c, ws, stream=cs)
+            forward(x_dev[cur], y_dev[cur], c, stream=cs)
             mb.moe_bias_update(dm, c, b, pid_state, params, stream=cs)
             comp_done[cur].record(cs)
             ds.wait_event(comp_done[cur])
@@ -446,7 +458,8 @@ def finish(args, w, world, rank, ms_max, routing, roof, layer, stage_ms, clk, e2
             "step": "moe_forward + moe_bias_update (PID target %.1f, kp=%g ki=%g kd=%g)"
                     % ((w.pid_target,) + PID_GAINS),
             "variant": {"renormalize_gates": bool(args.renormalize_gates),
-                        "balance_gamma": args.balance_gamma},
+                        "balance_gamma": args.balance_gamma,
+                        "expert_weights": "fp8 e4m3, 128x128 blocks" if args.fp8 else "bf16"},
             "mean_ffn_experts_per_token": round(float(np.mean(A_steps)) / w.T, 4),
             "distinct_ffn_experts": int(np.mean(U_steps)),
             "ffn_load_max_over_mean": round(float(np.mean(load_ratio)), 2),
@@ -524,6 +537,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg (profiling)")
     ap.add_argument("--renormalize-gates", action="store_true",
                     help="variant: gates renormalised over the K selected experts")
+    ap.add_argument("--fp8", action="store_true",
+                    help="variant: block-wise FP8 (E4M3) expert weights, quantised on the GPU")
     ap.add_argument("--balance-gamma", type=float, default=0.0,
                     help="variant: step of the per-expert balancing term after the PID step")
     args = ap.parse_args()

@@ -129,7 +129,8 @@ int moe_route(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *W_r, cons
  *   perm_tok  [T*K] int32   (out)   token of grouped row r (r < A)
  *   perm_gate [T*K] fp32    (out)   gate of grouped row r
  *   slot_pos  [T, K] int32  (out)   grouped row of slot (t, k), -1 for a zero-expert slot
- *   x_perm    [T*K, d] bf16 (out)   x_perm[r] = x[perm_tok[r]] for r < A
+ *   x_perm    [T*K, d] bf16 (out, nullable)  x_perm[r] = x[perm_tok[r]] for r < A; NULL skips
+ *                                   the copy (moe_expert_ffn_gather reads x directly)
  * Rows r >= A of the [T*K]-sized outputs are left untouched. */
 int moe_dispatch(const moe_dims *dims, const moe_bf16 *x, const int32_t *topk_idx,
                  const float *topk_gate, int32_t *counts, int32_t *offsets, int32_t *perm_tok,
@@ -164,6 +165,20 @@ int moe_expert_ffn(const moe_dims *dims, const moe_bf16 *x_perm, const int32_t *
                    const float *perm_gate, const moe_bf16 *W_g, const moe_bf16 *W_u,
                    const moe_bf16 *W_d, moe_bf16 *h, moe_bf16 *y_perm, void *ws,
                    size_t ws_bytes, void *stream);
+
+/* moe_expert_ffn with the dispatch gather fused into the up-projection: grouped row r's
+ * token row is read straight from x[perm_tok[r]] by the GEMM's loads (TMA row gathers), so no
+ * x_perm copy is written or read: T*K*d*2 bytes of memory saved, at a cost in speed (the
+ * row-by-row loads limit the up-projection; moe_forward keeps the copy).  Arguments as
+ * moe_expert_ffn, with
+ *   x        [T, d] bf16      the tokens (as given to moe_dispatch)
+ *   perm_tok [T*K] int32      token of each grouped row, from moe_dispatch (values in [0, T))
+ * in place of x_perm.  h and y_perm are bit-identical to moe_expert_ffn on the gathered
+ * x_perm. */
+int moe_expert_ffn_gather(const moe_dims *dims, const moe_bf16 *x, const int32_t *perm_tok,
+                          const int32_t *offsets, const float *perm_gate, const moe_bf16 *W_g,
+                          const moe_bf16 *W_u, const moe_bf16 *W_d, moe_bf16 *h,
+                          moe_bf16 *y_perm, void *ws, size_t ws_bytes, void *stream);
 
 /* Combine / un-permute: y_t = sum over FFN slots k (ascending expert id) of y_perm[slot_pos]
  * + (sum of the zero-expert gates of t) * x_t, accumulated in fp32 in that fixed order and
@@ -213,6 +228,41 @@ int moe_forward_timed(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *W
                       const float *b, const moe_bf16 *W_g, const moe_bf16 *W_u,
                       const moe_bf16 *W_d, moe_bf16 *y, int32_t *counts, void *ws,
                       size_t ws_bytes, void *const *stage_events, void *stream);
+
+/* ---------------------------------------------------------------- FP8 expert weights
+ * Block-wise FP8 quantisation ("衝上熱搜！美團大模型，靠「快」火了", §系統級優化: the same
+ * fine-grained block-wise scheme as DeepSeek-V3, one scale per 128 x 128 weight block).  For
+ * each of G matrices w[g] [R, C] and each 128 x 128 block: e = the smallest integer with
+ * max|w| <= 448 * 2^e (e >= -126; 0 for an all-zero block), scale = 2^e, and
+ * q = E4M3(w / 2^e), rounded to nearest with ties to even and saturated at +-448 (E4M3: 1 sign,
+ * 4 exponent bits biased by 7, 3 mantissa bits, S.1111.111 = NaN, largest finite 448).  The
+ * element format and the power-of-two scale are readings; with them q * scale is exact in
+ * bf16.
+ *   w     [G, R, C] bf16            R and C multiples of 128 (MOE_ERR_SHAPE otherwise)
+ *   q     [G, R, C] uint8 (out)     E4M3 codes
+ *   scale [G, R/128, C/128] fp32 (out)
+ * Expert weights: W_g and W_u with G = N, R = I, C = d; W_d with G = N, R = d, C = I. */
+int moe_quantize_fp8(const moe_bf16 *w, int64_t G, int64_t R, int64_t C, uint8_t *q,
+                     float *scale, void *stream);
+
+/* moe_expert_ffn with block-quantised expert weights (from moe_quantize_fp8): each weight
+ * tile is read as E4M3 codes (half the bytes of bf16) and turned into the exact bf16 weights
+ * q * scale in shared memory; activations, accumulation and outputs are as in moe_expert_ffn,
+ * so the result equals moe_expert_ffn on the dequantised weights.  d and I must be multiples
+ * of 128. */
+int moe_expert_ffn_fp8(const moe_dims *dims, const moe_bf16 *x_perm, const int32_t *offsets,
+                       const float *perm_gate, const uint8_t *q_g, const float *s_g,
+                       const uint8_t *q_u, const float *s_u, const uint8_t *q_d,
+                       const float *s_d, moe_bf16 *h, moe_bf16 *y_perm, void *ws,
+                       size_t ws_bytes, void *stream);
+
+/* moe_forward with block-quantised expert weights (the router weights stay bf16);
+ * stage_events as in moe_forward_timed, or NULL. */
+int moe_forward_fp8(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *W_r,
+                    const float *b, const uint8_t *q_g, const float *s_g, const uint8_t *q_u,
+                    const float *s_u, const uint8_t *q_d, const float *s_d, moe_bf16 *y,
+                    int32_t *counts, void *ws, size_t ws_bytes, void *const *stage_events,
+                    void *stream);
 
 /* Synchronises `stream`, returns the device status word of the workspace (MOE_DEV_* code,
  * 0 if none) and clears it.  Returns a negative value if the synchronisation itself failed. */

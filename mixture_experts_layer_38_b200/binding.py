@@ -18,7 +18,8 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 EXPORTS = (
     "moe_strerror", "moe_workspace_size", "moe_scratch_size", "moe_route", "moe_dispatch",
     "moe_expert_ffn", "moe_combine", "moe_bias_update", "moe_forward", "moe_forward_timed",
-    "moe_last_device_error", "moe_dispatch_noalloc",
+    "moe_last_device_error", "moe_dispatch_noalloc", "moe_expert_ffn_gather",
+    "moe_quantize_fp8", "moe_expert_ffn_fp8", "moe_forward_fp8",
 )
 NUM_STAGE_EVENTS = 7
 STAGE_NAMES = ("router_gemm", "route_topk", "dispatch", "ffn_up_gemm", "ffn_down_gemm",
@@ -80,9 +81,16 @@ def lib():
                                         ctypes.POINTER(ctypes.c_void_p), _P]
         L.moe_last_device_error.argtypes = [_P, _P]
         L.moe_dispatch_noalloc.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
+        L.moe_expert_ffn_gather.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]
+        _I64 = ctypes.c_int64
+        L.moe_quantize_fp8.argtypes = [_P, _I64, _I64, _I64, _P, _P, _P]
+        L.moe_expert_ffn_fp8.argtypes = [_DP] + [_P] * 11 + [_P, _S, _P]
+        L.moe_forward_fp8.argtypes = [_DP] + [_P] * 11 + [_P, _S,
+                                                          ctypes.POINTER(ctypes.c_void_p), _P]
         for f in ("moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine",
                   "moe_bias_update", "moe_forward", "moe_forward_timed",
-                  "moe_last_device_error", "moe_dispatch_noalloc"):
+                  "moe_last_device_error", "moe_dispatch_noalloc", "moe_expert_ffn_gather",
+                  "moe_quantize_fp8", "moe_expert_ffn_fp8", "moe_forward_fp8"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -171,7 +179,7 @@ def moe_dispatch(dm, x, topk_idx, topk_gate, counts, offsets, perm_tok, perm_gat
         _ptr(counts, torch.int32, (E,), "counts"), _ptr(offsets, torch.int32, (dm.N + 1,), "offsets"),
         _ptr(perm_tok, torch.int32, (R,), "perm_tok"), _ptr(perm_gate, torch.float32, (R,), "perm_gate"),
         _ptr(slot_pos, torch.int32, (dm.T, dm.K), "slot_pos"),
-        _ptr(x_perm, torch.bfloat16, (R, dm.d), "x_perm"), w, n, _stream(stream))
+        _ptr(x_perm, torch.bfloat16, (R, dm.d), "x_perm", nullable=True), w, n, _stream(stream))
     _check("moe_dispatch", rc)
 
 
@@ -204,6 +212,23 @@ def moe_expert_ffn(dm, x_perm, offsets, perm_gate, W_g, W_u, W_d, h, y_perm, ws,
         _ptr(h, torch.bfloat16, (R, dm.I), "h"), _ptr(y_perm, torch.bfloat16, (R, dm.d), "y_perm"),
         w, n, _stream(stream))
     _check("moe_expert_ffn", rc)
+
+
+def moe_expert_ffn_gather(dm, x, perm_tok, offsets, perm_gate, W_g, W_u, W_d, h, y_perm, ws,
+                          stream=None):
+    R = dm.T * dm.K
+    w, n = _ws(ws)
+    rc = lib().moe_expert_ffn_gather(
+        ctypes.byref(dm), _ptr(x, torch.bfloat16, (dm.T, dm.d), "x"),
+        _ptr(perm_tok, torch.int32, (R,), "perm_tok"),
+        _ptr(offsets, torch.int32, (dm.N + 1,), "offsets"),
+        _ptr(perm_gate, torch.float32, (R,), "perm_gate"),
+        _ptr(W_g, torch.bfloat16, (dm.N, dm.I, dm.d), "W_g"),
+        _ptr(W_u, torch.bfloat16, (dm.N, dm.I, dm.d), "W_u"),
+        _ptr(W_d, torch.bfloat16, (dm.N, dm.d, dm.I), "W_d"),
+        _ptr(h, torch.bfloat16, (R, dm.I), "h"), _ptr(y_perm, torch.bfloat16, (R, dm.d), "y_perm"),
+        w, n, _stream(stream))
+    _check("moe_expert_ffn_gather", rc)
 
 
 def moe_combine(dm, x, y_perm, topk_idx, topk_gate, slot_pos, y, stream=None):
@@ -262,3 +287,65 @@ def moe_forward_timed(dm, x, W_r, b, W_g, W_u, W_d, y, counts, ws, events, strea
 
 def moe_last_device_error(ws, stream=None) -> int:
     return int(lib().moe_last_device_error(_ptr(ws, torch.uint8, name="ws"), _stream(stream)))
+
+
+def moe_quantize_fp8(w, q, scale, stream=None):
+    """Block-wise E4M3 codes and power-of-two scales of bf16 weights [G, R, C] (or [R, C])."""
+    shape = tuple(w.shape) if w.dim() == 3 else (1,) + tuple(w.shape)
+    G, R, C = shape
+    rc = lib().moe_quantize_fp8(
+        _ptr(w, torch.bfloat16, tuple(w.shape), "w"), G, R, C,
+        _ptr(q, torch.uint8, tuple(w.shape), "q"),
+        _ptr(scale, torch.float32, (G, R // 128, C // 128) if w.dim() == 3 else
+             (R // 128, C // 128), "scale"), _stream(stream))
+    _check("moe_quantize_fp8", rc)
+
+
+def quantize_expert_weights_fp8(dm, W_g, W_u, W_d, stream=None):
+    """All three expert weight tensors quantised on the device: a dict of codes and scales."""
+    out = {}
+    for name, w in (("g", W_g), ("u", W_u), ("d", W_d)):
+        G, R, C = w.shape
+        out["q_" + name] = torch.empty((G, R, C), dtype=torch.uint8, device=w.device)
+        out["s_" + name] = torch.empty((G, R // 128, C // 128), dtype=torch.float32,
+                                       device=w.device)
+        moe_quantize_fp8(w, out["q_" + name], out["s_" + name], stream)
+    return out
+
+
+def _fp8_args(dm, fw):
+    I, d, N = dm.I, dm.d, dm.N
+    return (_ptr(fw["q_g"], torch.uint8, (N, I, d), "q_g"),
+            _ptr(fw["s_g"], torch.float32, (N, I // 128, d // 128), "s_g"),
+            _ptr(fw["q_u"], torch.uint8, (N, I, d), "q_u"),
+            _ptr(fw["s_u"], torch.float32, (N, I // 128, d // 128), "s_u"),
+            _ptr(fw["q_d"], torch.uint8, (N, d, I), "q_d"),
+            _ptr(fw["s_d"], torch.float32, (N, d // 128, I // 128), "s_d"))
+
+
+def moe_expert_ffn_fp8(dm, x_perm, offsets, perm_gate, fw, h, y_perm, ws, stream=None):
+    R = dm.T * dm.K
+    w, n = _ws(ws)
+    rc = lib().moe_expert_ffn_fp8(
+        ctypes.byref(dm), _ptr(x_perm, torch.bfloat16, (R, dm.d), "x_perm"),
+        _ptr(offsets, torch.int32, (dm.N + 1,), "offsets"),
+        _ptr(perm_gate, torch.float32, (R,), "perm_gate"), *_fp8_args(dm, fw),
+        _ptr(h, torch.bfloat16, (R, dm.I), "h"), _ptr(y_perm, torch.bfloat16, (R, dm.d), "y_perm"),
+        w, n, _stream(stream))
+    _check("moe_expert_ffn_fp8", rc)
+
+
+def moe_forward_fp8(dm, x, W_r, b, fw, y, counts, ws, stream=None, events=None):
+    w, n = _ws(ws)
+    ev = None
+    if events is not None:
+        assert len(events) == NUM_STAGE_EVENTS
+        ev = (ctypes.c_void_p * NUM_STAGE_EVENTS)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    rc = lib().moe_forward_fp8(
+        ctypes.byref(dm), _ptr(x, torch.bfloat16, (dm.T, dm.d), "x"),
+        _ptr(W_r, torch.bfloat16, (dm.N + dm.Z, dm.d), "W_r"),
+        _ptr(b, torch.float32, (dm.N + dm.Z,), "b"), *_fp8_args(dm, fw),
+        _ptr(y, torch.bfloat16, (dm.T, dm.d), "y"),
+        _ptr(counts, torch.int32, (dm.N + dm.Z,), "counts", nullable=True), w, n, ev,
+        _stream(stream))
+    _check("moe_forward_fp8", rc)

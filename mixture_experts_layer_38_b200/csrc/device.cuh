@@ -85,6 +85,26 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *m
       : "memory");
 }
 
+// Row-gather bulk copy (sm_100a): four rows r0..r3 of a 2-D tensor map whose box is 64
+// columns x 1 row, columns [c0, c0 + 64), land in shared memory as 4 consecutive 128-byte rows
+// (swizzled by destination address like a tiled load); completes 512 bytes on `bar`.
+__device__ __forceinline__ void tma_gather4(void *smem_dst, const CUtensorMap *map,
+                                            uint64_t *bar, int c0, int r0, int r1, int r2,
+                                            int r3, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1),
+      "r"(r2), "r"(r3), "l"(policy)
+      : "memory");
+}
+
+// Orders this thread's generic-proxy shared-memory stores before later async-proxy reads
+// (the tensor cores' operand fetches) of the same bytes.
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));

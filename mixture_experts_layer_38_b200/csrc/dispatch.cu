@@ -162,9 +162,10 @@ cudaError_t launch_dispatch(const uint16_t *x, const int32_t *topk_idx, const fl
     dispatch_permute_kernel<<<nchunks, kDispatchChunk, mask_bytes, stream>>>(
         topk_idx, topk_gate, T, K, N, E, chunk_counts, offsets, perm_tok, perm_gate, slot_pos,
         status);
-    gather_rows_kernel<<<num_sms * 8, 256, 0, stream>>>(
-        reinterpret_cast<const uint4 *>(x), d / 8, T, perm_tok, offsets + N,
-        reinterpret_cast<uint4 *>(x_perm), status);
+    if (x_perm != nullptr)  // NULL: the up-projection gathers the rows itself
+      gather_rows_kernel<<<num_sms * 8, 256, 0, stream>>>(
+          reinterpret_cast<const uint4 *>(x), d / 8, T, perm_tok, offsets + N,
+          reinterpret_cast<uint4 *>(x_perm), status);
   }
   return cudaGetLastError();
 }

@@ -32,6 +32,8 @@
 //
 // Every wait is bounded (device.cuh): on timeout the kernel records MOE_DEV_WAIT_TIMEOUT, all
 // roles unwind, in-flight copies and MMAs are drained (again bounded) and TMEM is freed.
+#include <cuda_fp8.h>
+
 #include "device.cuh"
 #include "kernels.cuh"
 
@@ -59,14 +61,27 @@ constexpr int kSmemPrefix = 2 * (kMaxGroups + 4) * 4;  // full-tile and tail-til
 // epilogue overlaps the next tile.  BN = 256: 64 KB stages, 3 in the ring, one 2 x 256-column
 // accumulator; every MMA and token load does twice the work, which is what compute-bound
 // tiles need (the issuing threads, not the tensor cores, limit 128-wide tiles).
-template <int BN>
+//
+// FP8 weights (WQ, used with BN = 128): a stage holds the two weight blocks as E4M3 codes
+// (2 x 8 KB, half the bytes, so twice the weights in flight per byte of ring) and the token
+// rows; eight converter warps (one block each per group of four) turn the codes into bf16
+// (times the block's power-of-two scale: exact) in a separate ring of two 32 KB bf16 slots,
+// which is what the MMA reads.  A stage is free again once the converters have read its
+// codes and the MMA its token rows; a slot once the MMA has read it.
+constexpr int kQTile = kBM * kBK;            // 8 KB of E4M3 codes per weight block
+constexpr int kConvWarps = 8;
+
+template <int BN, bool WQ = false>
 struct Cfg {
   static constexpr int kAccBufs = BN <= 128 ? 2 : 1;
-  static constexpr int kStage = 2 * kTileA + BN * kBK * 2;
-  static constexpr int kStages = (192 * 1024) / kStage;
-  static constexpr int kNumBars = 2 * kStages + 2 * kAccBufs + 1;
-  static constexpr int kSmemBytes =
-      1024 + kStages * kStage + kSmemStaging + kSmemPrefix + kNumBars * 8 + 16;
+  static constexpr int kStage = (WQ ? 2 * kQTile : 2 * kTileA) + BN * kBK * 2;
+  static constexpr int kCSlots = WQ ? 2 : 0;              // bf16 weight slots
+  static constexpr int kCRing = kCSlots * 2 * kTileA;
+  static constexpr int kStages = (192 * 1024 - kCRing) / kStage;
+  static constexpr int kNumBars = 2 * kStages + 2 * kAccBufs + 1 + 2 * kCSlots;
+  static constexpr int kThreads = 64 + 32 * kEpiWarps + (WQ ? 32 * kConvWarps : 0);
+  static constexpr int kSmemBytes = 1024 + kStages * kStage + kCRing + kSmemStaging +
+                                    kSmemPrefix + kNumBars * 8 + 16;
   static_assert(kAccBufs * 2 * BN <= kTmemCols, "TMEM holds 512 columns");
   static_assert(kSmemBytes <= 232448, "shared memory per block");
 };
@@ -170,7 +185,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *scratch, int &to
   __syncthreads();
   int base = 0;
   total = 0;
-  for (int w = 0; w < kGemmThreads / 32; ++w) {
+  for (int w = 0; w < (int)(blockDim.x / 32); ++w) {
     if (w < warp) base += scratch[w];
     total += scratch[w];
   }
@@ -184,7 +199,7 @@ template <int BN>
 __device__ bool build_schedule(const GemmArgs &a, int *hpre, int *lpre, int *scratch,
                                Schedule &s) {
   const int G = a.group_offsets ? a.num_groups : 1;
-  const int per = (G + kGemmThreads - 1) / kGemmThreads;
+  const int per = (G + (int)blockDim.x - 1) / (int)blockDim.x;
   const int g_begin = min(G, (int)threadIdx.x * per);
   const int g_end = min(G, g_begin + per);
   int nh = 0, nl = 0;
@@ -331,15 +346,46 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs &a, const Tile &t,
   }
 }
 
-template <int EPI, int BN>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+// E4M3 block (128 rows x 64 codes, row-major) -> bf16 block in the 128-byte-swizzled K-major
+// layout the MMA descriptors read, times `scale` (a power of two: exact).  `ct` in [0, 128):
+// each thread converts one 16-code chunk of a row per pass; consecutive threads read
+// consecutive 16-byte chunks, and each warp's stores cover all 32 banks four times.
+__device__ __forceinline__ void convert_fp8_block(const uint8_t *q, uint8_t *dst, float scale,
+                                                  int ct) {
+#pragma unroll
+  for (int pass = 0; pass < 4; ++pass) {
+    const int r = pass * 32 + (ct >> 2), c = ct & 3;
+    const uint4 v = *reinterpret_cast<const uint4 *>(q + r * kBK + c * 16);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(
+            static_cast<__nv_fp8x2_storage_t>((w[i] >> (16 * h)) & 0xffffu), __NV_E4M3);
+        const float2 f = __half22float2(__half2(hr));
+        const __nv_bfloat162 b = __floats2bfloat162_rn(f.x * scale, f.y * scale);
+        o[2 * i + h] = *reinterpret_cast<const uint32_t *>(&b);
+      }
+    }
+    uint8_t *row = dst + r * (kBK * 2);
+    const int j0 = 2 * c, sw = r & 7;
+    *reinterpret_cast<uint4 *>(row + ((j0 ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4 *>(row + (((j0 + 1) ^ sw) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
+template <int EPI, int BN, bool WQ, bool GATHER>
+__global__ void __launch_bounds__(Cfg<BN, WQ>::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ GemmArgs args) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, WQ>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t *ring = smem;
-  constexpr int kRing = C::kStages * C::kStage;
+  constexpr int kRing = C::kStages * C::kStage + C::kCRing;
+  uint8_t *cring = smem + C::kStages * C::kStage;  // WQ: bf16 weight slots (2 x 16 KB each)
   float *staging = reinterpret_cast<float *>(smem + kRing);
   int *hpre = reinterpret_cast<int *>(smem + kRing + kSmemStaging);
   int *lpre = hpre + kMaxGroups + 4;
@@ -349,6 +395,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t *tfull_bar = bars + 2 * C::kStages;
   uint64_t *tempty_bar = bars + 2 * C::kStages + C::kAccBufs;
   uint64_t *drain_bar = bars + 2 * C::kStages + 2 * C::kAccBufs;
+  uint64_t *cfull_bar = drain_bar + 1;           // WQ: slot holds converted weights
+  uint64_t *cempty_bar = cfull_bar + C::kCSlots;  // WQ: the MMA has read the slot
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::kNumBars);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -358,13 +406,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], 1);
+      mbar_init(&empty_bar[s], WQ ? 1 + kConvWarps : 1);  // WQ: the converters read it too
     }
     for (int b = 0; b < C::kAccBufs; ++b) {
       mbar_init(&tfull_bar[b], 1);
       mbar_init(&tempty_bar[b], kEpiWarps);
     }
     mbar_init(drain_bar, 1);
+    for (int c = 0; c < C::kCSlots; ++c) {
+      mbar_init(&cfull_bar[c], kConvWarps);
+      mbar_init(&cempty_bar[c], 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -375,6 +427,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tma_prefetch_desc(&args.map_b256);
 #pragma unroll
     for (int i = 0; i < 4; ++i) tma_prefetch_desc(&args.map_b[i]);
+    if (GATHER) tma_prefetch_desc(&args.map_bg);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -392,7 +445,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
-    if (lane == 0) {
+    // Lane 0 issues the weight loads and the tiled token loads.  In gather mode the whole warp
+    // runs the loop and every lane issues tile::gather4 loads of 4 token rows each (groups
+    // `lane` and `lane + 32` of the tile's nb rows) after lane 0 has armed the stage's barrier.
+    constexpr bool gather = GATHER;
+    if (gather || lane == 0) {
       // Weights of a group with a single token tile are read once: stream them past L2
       // (evict-first) so they do not push out the tiles other CTAs are still re-reading.
       const uint64_t pol_w_reused = l2_policy_evict_normal();
@@ -404,48 +461,76 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < sched.total; tile += gridDim.x) {
         const Tile t = decode_tile<EPI, BN>(args, sched, tile);
-        const uint32_t bytes = kTileA * (t.has_a1 ? 2 : 1) + t.nb * kBK * 2;
+        const uint32_t bytes = (WQ ? kQTile : kTileA) * (t.has_a1 ? 2 : 1) + t.nb * kBK * 2;
         const uint64_t pol_w = t.once ? pol_w_once : pol_w_reused;
+        int rix[8];  // gather mode: source rows of this lane's two 4-row groups
+        if (gather) {
+  #pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int r = (i < 4 ? lane : lane + 32) * 4 + (i & 3);
+            rix[i] = __ldg(args.row_index + t.row0 + min(r, t.n_valid - 1));  // pad: a valid row
+          }
+        }
+        const int groups = t.nb >> 2;
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
-          if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag)) {
-            signal_abort(args, abort_flag);
+          if (!(gather ? warp_wait(&empty_bar[stage], phase ^ 1, abort_flag)
+                       : mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag))) {
+            if (lane == 0) signal_abort(args, abort_flag);
             ok = false;
             break;
           }
           uint8_t *sa0 = ring + stage * C::kStage;
           uint8_t *sa1 = sa0 + kTileA;
-          uint8_t *sb = sa0 + 2 * kTileA;
+          uint8_t *sb = sa0 + (WQ ? 2 * kQTile : 2 * kTileA);
           const int kc = kb * kBK;
-          mbar_arrive_expect_tx(&full_bar[stage], bytes);
-          if (kWideBoxes && EPI != kEpiSwiGLU && t.has_a1) {
-            tma_load_2d(sa0, &args.map_a01, &full_bar[stage], kc, t.a0_row, pol_w);
-          } else {
-            tma_load_2d(sa0, &args.map_a0, &full_bar[stage], kc, t.a0_row, pol_w);
-            if (t.has_a1) tma_load_2d(sa1, &args.map_a1, &full_bar[stage], kc, t.a1_row, pol_w);
-          }
-          // Token rows in boxes of 256 / 128 (as many as needed), then 64 / 32 / 16.
-          int r = 0;
-          if (kWideBoxes && t.nb == 256) {
-            tma_load_2d(sb, &args.map_b256, &full_bar[stage], kc, t.row0, pol_x);
-            r = 256;
-          }
-          for (; t.nb - r >= 128; r += 128)
-            tma_load_2d(sb + r * (kBK * 2), &args.map_b[0], &full_bar[stage], kc, t.row0 + r,
-                        pol_x);
-#pragma unroll
-          for (int i = 1; i < 4; ++i) {
-            const int box = 128 >> i;
-            if (t.nb - r >= box) {
-              tma_load_2d(sb + r * (kBK * 2), &args.map_b[i], &full_bar[stage], kc, t.row0 + r,
-                          pol_x);
-              r += box;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&full_bar[stage], bytes);
+            if (WQ) {  // E4M3 codes of both weight blocks at the start of the stage
+              tma_load_2d(sa0, &args.map_a0, &full_bar[stage], kc, t.a0_row, pol_w);
+              if (t.has_a1)
+                tma_load_2d(sa0 + kQTile, &args.map_a1, &full_bar[stage], kc, t.a1_row, pol_w);
+            } else if (kWideBoxes && EPI != kEpiSwiGLU && t.has_a1) {
+              tma_load_2d(sa0, &args.map_a01, &full_bar[stage], kc, t.a0_row, pol_w);
+            } else {
+              tma_load_2d(sa0, &args.map_a0, &full_bar[stage], kc, t.a0_row, pol_w);
+              if (t.has_a1)
+                tma_load_2d(sa1, &args.map_a1, &full_bar[stage], kc, t.a1_row, pol_w);
             }
+            if (!gather) {
+              // Token rows in boxes of 256 / 128 (as many as needed), then 64 / 32 / 16.
+              int r = 0;
+              if (kWideBoxes && t.nb == 256) {
+                tma_load_2d(sb, &args.map_b256, &full_bar[stage], kc, t.row0, pol_x);
+                r = 256;
+              }
+              for (; t.nb - r >= 128; r += 128)
+                tma_load_2d(sb + r * (kBK * 2), &args.map_b[0], &full_bar[stage], kc,
+                            t.row0 + r, pol_x);
+#pragma unroll
+              for (int i = 1; i < 4; ++i) {
+                const int box = 128 >> i;
+                if (t.nb - r >= box) {
+                  tma_load_2d(sb + r * (kBK * 2), &args.map_b[i], &full_bar[stage], kc,
+                              t.row0 + r, pol_x);
+                  r += box;
+                }
+              }
+            }
+          }
+          if (gather) {
+            __syncwarp();  // the barrier is armed before any gathered bytes can land
+            if (lane < groups)
+              tma_gather4(sb + lane * (4 * kBK * 2), &args.map_bg, &full_bar[stage], kc, rix[0],
+                          rix[1], rix[2], rix[3], pol_x);
+            if (lane + 32 < groups)
+              tma_gather4(sb + (lane + 32) * (4 * kBK * 2), &args.map_bg, &full_bar[stage], kc,
+                          rix[4], rix[5], rix[6], rix[7], pol_x);
           }
           ++issued;
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
         }
       }
-      if (!ok) {
+      if (!ok && lane == 0) {
         // Drain the copies that may still be landing in the ring (bounded).
         for (long long i = 1; i <= issued && i <= C::kStages; ++i) {
           const long long idx = issued - i;
@@ -461,6 +546,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      int cslot = 0;            // WQ: bf16 slot of the current k-step
+      uint32_t cphase = 0;
       int it = 0;
       bool ok = true;
       bool any = false;
@@ -478,23 +565,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const uint32_t d1 = d0 + BN;
         const uint32_t idesc = idesc_bf16_f32(kBM, t.nb);
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
-          if (!mbar_wait(&full_bar[stage], phase, abort_flag)) {
+          if (!mbar_wait(&full_bar[stage], phase, abort_flag) ||
+              (WQ && !mbar_wait(&cfull_bar[cslot], cphase, abort_flag))) {
             signal_abort(args, abort_flag);
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t base = smem_u32(ring + stage * C::kStage);
+          const uint32_t sbase = smem_u32(ring + stage * C::kStage);
+          const uint32_t abase = WQ ? smem_u32(cring + cslot * (2 * kTileA)) : sbase;
+          const uint32_t bbase = sbase + (WQ ? 2 * kQTile : 2 * kTileA);
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k) {
-            const uint64_t bdesc = sw128_kmajor_desc(base + 2 * kTileA + k * 32);
+            const uint64_t bdesc = sw128_kmajor_desc(bbase + k * 32);
             const uint32_t acc = (kb > t.kb0 || k > 0) ? 1u : 0u;
-            umma_bf16(d0, sw128_kmajor_desc(base + k * 32), bdesc, idesc, acc);
-            if (t.has_a1) umma_bf16(d1, sw128_kmajor_desc(base + kTileA + k * 32), bdesc, idesc, acc);
+            umma_bf16(d0, sw128_kmajor_desc(abase + k * 32), bdesc, idesc, acc);
+            if (t.has_a1)
+              umma_bf16(d1, sw128_kmajor_desc(abase + kTileA + k * 32), bdesc, idesc, acc);
           }
           any = true;
           umma_commit(&empty_bar[stage]);
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+          if (WQ) {
+            umma_commit(&cempty_bar[cslot]);
+            if (++cslot == C::kCSlots) { cslot = 0; cphase ^= 1; }
+          }
         }
         if (!ok) break;
         umma_commit(&tfull_bar[buf]);
@@ -503,6 +598,41 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         umma_commit(drain_bar);
         const long long t0 = clock64();
         while (!mbar_try_wait(drain_bar, 0) && clock64() - t0 < kDrainLimitCycles) {}
+      }
+    }
+  } else if (WQ && warp >= 2 + kEpiWarps) {
+    // ---------------------------------------------------------------- converters (FP8)
+    // Warps 0-3 of the converters handle weight block 0 of each k-step, warps 4-7 block 1.
+    const int ct = (int)threadIdx.x - (2 + kEpiWarps) * 32;
+    const int half = ct >> 7, lt = ct & 127;
+    int stage = 0, cslot = 0;
+    uint32_t phase = 0, cphase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < sched.total; tile += gridDim.x) {
+      const Tile t = decode_tile<EPI, BN>(args, sched, tile);
+      const int row = half ? t.a1_row : t.a0_row;
+      const float *scales = (half ? args.scale_a1 : args.scale_a0) + (row / 128) * args.scale_ld;
+      const bool mine = half == 0 || t.has_a1;
+      for (int kb = t.kb0; kb < t.kb1; ++kb) {
+        if (!warp_wait(&full_bar[stage], phase, abort_flag) ||
+            !warp_wait(&cempty_bar[cslot], cphase ^ 1, abort_flag)) {
+          if (lane == 0) signal_abort(args, abort_flag);
+          ok = false;
+          break;
+        }
+        if (mine) {
+          const uint8_t *q = ring + stage * C::kStage + half * kQTile;
+          uint8_t *dst = cring + cslot * (2 * kTileA) + half * kTileA;
+          convert_fp8_block(q, dst, __ldg(scales + (kb * kBK) / 128), lt);
+          fence_proxy_async_shared();  // generic-proxy stores -> visible to the tensor cores
+        }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&cfull_bar[cslot]);
+          mbar_arrive(&empty_bar[stage]);  // this warp is done reading the stage's codes
+        }
+        if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+        if (++cslot == C::kCSlots) { cslot = 0; cphase ^= 1; }
       }
     }
   } else {
@@ -538,24 +668,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
-template <int EPI, int BN>
+template <int EPI, int BN, bool WQ = false, bool GATHER = false>
 cudaError_t set_smem_limit() {
-  return cudaFuncSetAttribute(grouped_gemm_kernel<EPI, BN>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<BN>::kSmemBytes);
+  return cudaFuncSetAttribute(grouped_gemm_kernel<EPI, BN, WQ, GATHER>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              Cfg<BN, WQ>::kSmemBytes);
 }
 
 template <int BN>
 cudaError_t launch_bn(int epi, const GemmArgs &args, int grid, cudaStream_t stream) {
   constexpr int smem = Cfg<BN>::kSmemBytes;
+  constexpr int threads = Cfg<BN>::kThreads;
   switch (epi) {
     case kEpiSwiGLU:
-      grouped_gemm_kernel<kEpiSwiGLU, BN><<<grid, kGemmThreads, smem, stream>>>(args);
+      if (args.row_index != nullptr)
+        grouped_gemm_kernel<kEpiSwiGLU, BN, false, true><<<grid, threads, smem, stream>>>(args);
+      else
+        grouped_gemm_kernel<kEpiSwiGLU, BN, false, false><<<grid, threads, smem, stream>>>(args);
       break;
     case kEpiGated:
-      grouped_gemm_kernel<kEpiGated, BN><<<grid, kGemmThreads, smem, stream>>>(args);
+      grouped_gemm_kernel<kEpiGated, BN, false, false><<<grid, threads, smem, stream>>>(args);
       break;
     default:
-      grouped_gemm_kernel<kEpiF32, BN><<<grid, kGemmThreads, smem, stream>>>(args);
+      grouped_gemm_kernel<kEpiF32, BN, false, false><<<grid, threads, smem, stream>>>(args);
       break;
   }
   return cudaGetLastError();
@@ -571,6 +706,10 @@ cudaError_t gemm_prepare(int device) {
   if ((e = set_smem_limit<kEpiF32, 128>()) != cudaSuccess) return e;
   if ((e = set_smem_limit<kEpiSwiGLU, 256>()) != cudaSuccess) return e;
   if ((e = set_smem_limit<kEpiGated, 256>()) != cudaSuccess) return e;
+  if ((e = set_smem_limit<kEpiSwiGLU, 128, false, true>()) != cudaSuccess) return e;
+  if ((e = set_smem_limit<kEpiSwiGLU, 256, false, true>()) != cudaSuccess) return e;
+  if ((e = set_smem_limit<kEpiSwiGLU, 128, true>()) != cudaSuccess) return e;
+  if ((e = set_smem_limit<kEpiGated, 128, true>()) != cudaSuccess) return e;
   return set_smem_limit<kEpiF32, 256>();
 }
 
@@ -585,6 +724,20 @@ cudaError_t launch_grouped_gemm(int epi, const GemmArgs &args, int grid, int til
                                 cudaStream_t stream) {
   return tile_tokens == 256 ? launch_bn<256>(epi, args, grid, stream)
                             : launch_bn<128>(epi, args, grid, stream);
+}
+
+cudaError_t launch_grouped_gemm_fp8(int epi, const GemmArgs &args, int grid,
+                                    cudaStream_t stream) {
+  using C = Cfg<128, true>;
+  if (epi == kEpiSwiGLU)
+    grouped_gemm_kernel<kEpiSwiGLU, 128, true, false>
+        <<<grid, C::kThreads, C::kSmemBytes, stream>>>(args);
+  else if (epi == kEpiGated)
+    grouped_gemm_kernel<kEpiGated, 128, true, false>
+        <<<grid, C::kThreads, C::kSmemBytes, stream>>>(args);
+  else
+    return cudaErrorInvalidValue;
+  return cudaGetLastError();
 }
 
 }  // namespace moe

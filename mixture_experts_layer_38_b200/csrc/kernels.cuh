@@ -34,6 +34,17 @@ struct GemmArgs {
   long long split_stride;        // elements between split-K partial outputs
   const float *row_scale;        // kEpiGated: per-row gate
   int *status;                   // device status word
+  // Row gather (up-projection only): when row_index is set, activation row r is row
+  // row_index[r] of the matrix behind map_bg (64 x 1 boxes), fetched with tile::gather4;
+  // map_b / map_b256 are then unused.
+  const int *row_index;
+  CUtensorMap map_bg;
+  // FP8 weights (launch_grouped_gemm_fp8): map_a0 / map_a1 cover E4M3 codes (64 x 128 boxes,
+  // no swizzle); the scale of the 128 x 128 block holding weight row r, column k is
+  // scale_a0/1[(r / 128) * scale_ld + k / 128].
+  const float *scale_a0;
+  const float *scale_a1;
+  int scale_ld;
 };
 
 // Grouped GEMM block: warp 0 issues TMA loads, warp 1 allocates TMEM and issues MMAs, and
@@ -47,6 +58,14 @@ cudaError_t gemm_prepare(int device);  // sets the kernels' shared-memory limit 
 int gemm_tile_tokens(long long rows, int groups, int K);
 cudaError_t launch_grouped_gemm(int epi, const GemmArgs &args, int grid, int tile_tokens,
                                 cudaStream_t stream);
+// SwiGLU or gated grouped GEMM with E4M3 block-quantised weights, 128-token tiles.
+cudaError_t launch_grouped_gemm_fp8(int epi, const GemmArgs &args, int grid,
+                                    cudaStream_t stream);
+
+// Block-wise E4M3 of G matrices [R, C] bf16 (R, C multiples of 128): codes and one power-of-two
+// scale per 128 x 128 block.
+cudaError_t launch_quantize_fp8(const uint16_t *w, long long G, long long R, long long C,
+                                uint8_t *q, float *scale, cudaStream_t stream);
 
 // ------------------------------------------------------------------ routing
 // logits [splits][T][E] fp32 -> softmax, biased top-K, ascending ids.

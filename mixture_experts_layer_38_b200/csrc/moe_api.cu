@@ -86,6 +86,28 @@ bool make_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
          CUDA_SUCCESS;
 }
 
+// Row-major E4M3 codes [rows, cols] in boxes of 64 columns (64 bytes) x 128 rows, no swizzle
+// (the converter warps read them row by row).
+bool make_map_u8(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estride[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box,
+            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+// Block-quantised expert weights: E4M3 codes in the bf16 weights' layouts and one fp32
+// power-of-two scale per 128 x 128 block ([N][rows / 128][cols / 128]).
+struct Fp8Weights {
+  const uint8_t *q_g, *q_u, *q_d;
+  const float *s_g, *s_u, *s_d;
+};
+
 bool make_act_maps(GemmArgs &a, const void *base, uint64_t rows, uint64_t cols) {
   for (int i = 0; i < 4; ++i)
     if (!make_map(&a.map_b[i], base, rows, cols, 128u >> i)) return false;
@@ -106,6 +128,9 @@ bool dims_ok(const moe_dims *d) {
   if ((d->flags & ~MOE_RENORMALIZE_GATES) != 0) return false;
   return true;
 }
+
+// The FP8 weight path scales 128 x 128 blocks: both GEMMs' dims must be whole blocks.
+bool fp8_dims_ok(const moe_dims &d) { return d.d % 128 == 0 && d.I % 128 == 0; }
 
 int router_splits(const moe_dims &d) {
   const int E = d.N + d.Z;
@@ -250,17 +275,27 @@ int do_expert_ffn(const moe_dims &d, const DeviceInfo &di, const Layout &L,
                   const moe_bf16 *x_perm, const int32_t *offsets, const float *perm_gate,
                   const moe_bf16 *W_g, const moe_bf16 *W_u, const moe_bf16 *W_d, moe_bf16 *h,
                   moe_bf16 *y_perm, void *ws, cudaStream_t stream,
-                  void *const *events = nullptr) {
+                  void *const *events = nullptr, const moe_bf16 *x = nullptr,
+                  const int32_t *perm_tok = nullptr, const Fp8Weights *fw = nullptr) {
   if (d.T == 0 || d.N == 0) return record(events, 4, stream);
   const uint64_t rows = (uint64_t)d.T * d.K;
   int *status = at<int>(ws, L.status);
   GemmArgs up{};
-  if (!make_map(&up.map_a0, W_g, (uint64_t)d.N * d.I, (uint64_t)d.d, 128) ||
-      !make_map(&up.map_a1, W_u, (uint64_t)d.N * d.I, (uint64_t)d.d, 128) ||
-      !make_map(&up.map_a01, W_g, (uint64_t)d.N * d.I, (uint64_t)d.d, 256) ||
-      !make_act_maps(up, x_perm, rows, (uint64_t)d.d)) {
+  // Token rows: the grouped copy x_perm, or (perm_tok given) gathered from x by the GEMM.
+  const bool gather = perm_tok != nullptr;
+  const bool ok_w = fw != nullptr
+      ? make_map_u8(&up.map_a0, fw->q_g, (uint64_t)d.N * d.I, (uint64_t)d.d) &&
+            make_map_u8(&up.map_a1, fw->q_u, (uint64_t)d.N * d.I, (uint64_t)d.d) &&
+            make_map_u8(&up.map_a01, fw->q_g, (uint64_t)d.N * d.I, (uint64_t)d.d)
+      : make_map(&up.map_a0, W_g, (uint64_t)d.N * d.I, (uint64_t)d.d, 128) &&
+            make_map(&up.map_a1, W_u, (uint64_t)d.N * d.I, (uint64_t)d.d, 128) &&
+            make_map(&up.map_a01, W_g, (uint64_t)d.N * d.I, (uint64_t)d.d, 256);
+  if (!ok_w ||
+      !make_act_maps(up, gather ? x : x_perm, gather ? (uint64_t)d.T : rows, (uint64_t)d.d) ||
+      (gather && !make_map(&up.map_bg, x, (uint64_t)d.T, (uint64_t)d.d, 1))) {
     return MOE_ERR_CUDA;
   }
+  up.row_index = perm_tok;
   up.group_offsets = offsets;
   up.num_groups = d.N;
   up.rows = (int)rows;
@@ -272,16 +307,27 @@ int do_expert_ffn(const moe_dims &d, const DeviceInfo &di, const Layout &L,
   up.split_stride = 0;
   up.row_scale = nullptr;
   up.status = status;
+  if (fw != nullptr) {
+    up.scale_a0 = fw->s_g;
+    up.scale_a1 = fw->s_u;
+    up.scale_ld = d.d / 128;
+  }
   const int tile_tokens = gemm_tile_tokens((long long)rows, d.N, d.d);
-  if (launch_grouped_gemm(kEpiSwiGLU, up, di.sms, tile_tokens, stream) != cudaSuccess)
+  if ((fw != nullptr ? launch_grouped_gemm_fp8(kEpiSwiGLU, up, di.sms, stream)
+                     : launch_grouped_gemm(kEpiSwiGLU, up, di.sms, tile_tokens, stream)) !=
+      cudaSuccess)
     return MOE_ERR_CUDA;
   if (record(events, 4, stream) != MOE_OK) return MOE_ERR_CUDA;
 
   GemmArgs down{};
-  if (!make_map(&down.map_a0, W_d, (uint64_t)d.N * d.d, (uint64_t)d.I, 128) ||
-      !make_map(&down.map_a1, W_d, (uint64_t)d.N * d.d, (uint64_t)d.I, 128) ||
-      !make_map(&down.map_a01, W_d, (uint64_t)d.N * d.d, (uint64_t)d.I, 256) ||
-      !make_act_maps(down, h, rows, (uint64_t)d.I)) {
+  const bool ok_wd = fw != nullptr
+      ? make_map_u8(&down.map_a0, fw->q_d, (uint64_t)d.N * d.d, (uint64_t)d.I) &&
+            make_map_u8(&down.map_a1, fw->q_d, (uint64_t)d.N * d.d, (uint64_t)d.I) &&
+            make_map_u8(&down.map_a01, fw->q_d, (uint64_t)d.N * d.d, (uint64_t)d.I)
+      : make_map(&down.map_a0, W_d, (uint64_t)d.N * d.d, (uint64_t)d.I, 128) &&
+            make_map(&down.map_a1, W_d, (uint64_t)d.N * d.d, (uint64_t)d.I, 128) &&
+            make_map(&down.map_a01, W_d, (uint64_t)d.N * d.d, (uint64_t)d.I, 256);
+  if (!ok_wd || !make_act_maps(down, h, rows, (uint64_t)d.I)) {
     return MOE_ERR_CUDA;
   }
   down.group_offsets = offsets;
@@ -295,6 +341,12 @@ int do_expert_ffn(const moe_dims &d, const DeviceInfo &di, const Layout &L,
   down.split_stride = 0;
   down.row_scale = perm_gate;
   down.status = status;
+  if (fw != nullptr) {
+    down.scale_a0 = fw->s_d;
+    down.scale_a1 = fw->s_d;
+    down.scale_ld = d.I / 128;
+    return to_status(launch_grouped_gemm_fp8(kEpiGated, down, di.sms, stream));
+  }
   return to_status(launch_grouped_gemm(kEpiGated, down, di.sms, tile_tokens, stream));
 }
 
@@ -364,7 +416,7 @@ int moe_dispatch(const moe_dims *dims, const moe_bf16 *x, const int32_t *topk_id
   MOE_CHECK_TOKEN_PTR(perm_tok, dims->T);
   MOE_CHECK_TOKEN_PTR(perm_gate, dims->T);
   MOE_CHECK_TOKEN_PTR(slot_pos, dims->T);
-  MOE_CHECK_TOKEN_PTR(x_perm, dims->T);
+  if (x_perm != nullptr) MOE_REQUIRE(aligned16(x_perm), MOE_ERR_ALIGN);
   const Layout L = layout_of(*dims);
   int rc = check_ws(ws, ws_bytes, L.scratch_end);
   if (rc != MOE_OK) return rc;
@@ -397,6 +449,31 @@ int moe_expert_ffn(const moe_dims *dims, const moe_bf16 *x_perm, const int32_t *
   if (rc != MOE_OK) return rc;
   return do_expert_ffn(*dims, *di, L, x_perm, offsets, perm_gate, W_g, W_u, W_d, h, y_perm, ws,
                        static_cast<cudaStream_t>(stream));
+}
+
+int moe_expert_ffn_gather(const moe_dims *dims, const moe_bf16 *x, const int32_t *perm_tok,
+                          const int32_t *offsets, const float *perm_gate, const moe_bf16 *W_g,
+                          const moe_bf16 *W_u, const moe_bf16 *W_d, moe_bf16 *h,
+                          moe_bf16 *y_perm, void *ws, size_t ws_bytes, void *stream) {
+  MOE_REQUIRE(dims != nullptr, MOE_ERR_ARG);
+  MOE_REQUIRE(dims_ok(dims), MOE_ERR_SHAPE);
+  MOE_CHECK_TOKEN_PTR(x, dims->T);
+  MOE_CHECK_TOKEN_PTR(perm_tok, dims->T);
+  MOE_CHECK_PTR(offsets);
+  MOE_CHECK_TOKEN_PTR(perm_gate, dims->T);
+  MOE_CHECK_PTR(W_g);
+  MOE_CHECK_PTR(W_u);
+  MOE_CHECK_PTR(W_d);
+  MOE_CHECK_TOKEN_PTR(h, dims->T);
+  MOE_CHECK_TOKEN_PTR(y_perm, dims->T);
+  const Layout L = layout_of(*dims);
+  int rc = check_ws(ws, ws_bytes, L.scratch_end);
+  if (rc != MOE_OK) return rc;
+  const DeviceInfo *di = nullptr;
+  rc = device_info(&di);
+  if (rc != MOE_OK) return rc;
+  return do_expert_ffn(*dims, *di, L, nullptr, offsets, perm_gate, W_g, W_u, W_d, h, y_perm, ws,
+                       static_cast<cudaStream_t>(stream), nullptr, x, perm_tok);
 }
 
 int moe_combine(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *y_perm,
@@ -440,15 +517,26 @@ namespace {
 
 int forward_impl(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *W_r, const float *b,
                  const moe_bf16 *W_g, const moe_bf16 *W_u, const moe_bf16 *W_d, moe_bf16 *y,
-                 int32_t *counts, void *ws, size_t ws_bytes, void *const *ev, void *stream) {
+                 int32_t *counts, void *ws, size_t ws_bytes, void *const *ev, void *stream,
+                 const Fp8Weights *fw = nullptr) {
   MOE_REQUIRE(dims != nullptr, MOE_ERR_ARG);
   MOE_REQUIRE(dims_ok(dims), MOE_ERR_SHAPE);
   MOE_CHECK_TOKEN_PTR(x, dims->T);
   MOE_CHECK_PTR(W_r);
   MOE_CHECK_PTR(b);
-  MOE_CHECK_PTR(W_g);
-  MOE_CHECK_PTR(W_u);
-  MOE_CHECK_PTR(W_d);
+  if (fw == nullptr) {
+    MOE_CHECK_PTR(W_g);
+    MOE_CHECK_PTR(W_u);
+    MOE_CHECK_PTR(W_d);
+  } else {
+    MOE_REQUIRE(fp8_dims_ok(*dims), MOE_ERR_SHAPE);
+    MOE_CHECK_PTR(fw->q_g);
+    MOE_CHECK_PTR(fw->q_u);
+    MOE_CHECK_PTR(fw->q_d);
+    MOE_CHECK_PTR(fw->s_g);
+    MOE_CHECK_PTR(fw->s_u);
+    MOE_CHECK_PTR(fw->s_d);
+  }
   MOE_CHECK_TOKEN_PTR(y, dims->T);
   if (counts != nullptr) MOE_REQUIRE(aligned16(counts), MOE_ERR_ALIGN);
   if (ev != nullptr)
@@ -475,11 +563,14 @@ int forward_impl(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *W_r, c
   rc = do_route(d, *di, L, x, W_r, b, topk_idx, topk_gate, at<float>(ws, L.gap), ws, s, ev);
   if (rc != MOE_OK) return rc;
   if ((rc = record(ev, 2, s)) != MOE_OK) return rc;
+  // The gathered copy x_perm and tiled token loads: faster than gathering rows inside the
+  // up-projection (moe_expert_ffn_gather), whose row-by-row loads limit the GEMM.
   rc = do_dispatch(d, *di, L, x, topk_idx, topk_gate, cnt, offsets, perm_tok, perm_gate,
                    slot_pos, x_perm, ws, s);
   if (rc != MOE_OK) return rc;
   if ((rc = record(ev, 3, s)) != MOE_OK) return rc;
-  rc = do_expert_ffn(d, *di, L, x_perm, offsets, perm_gate, W_g, W_u, W_d, h, y_perm, ws, s, ev);
+  rc = do_expert_ffn(d, *di, L, x_perm, offsets, perm_gate, W_g, W_u, W_d, h, y_perm, ws, s, ev,
+                     nullptr, nullptr, fw);
   if (rc != MOE_OK) return rc;
   if ((rc = record(ev, 5, s)) != MOE_OK) return rc;
   rc = to_status(launch_combine(x, y_perm, topk_idx, topk_gate, slot_pos, d.T, d.d, d.N, d.K,
@@ -505,6 +596,61 @@ int moe_forward_timed(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *W
   MOE_REQUIRE(stage_events != nullptr, MOE_ERR_ARG);
   return forward_impl(dims, x, W_r, b, W_g, W_u, W_d, y, counts, ws, ws_bytes, stage_events,
                       stream);
+}
+
+int moe_quantize_fp8(const moe_bf16 *w, int64_t G, int64_t R, int64_t C, uint8_t *q,
+                     float *scale, void *stream) {
+  MOE_REQUIRE(G >= 0 && R >= 0 && C >= 0 && R % 128 == 0 && C % 128 == 0, MOE_ERR_SHAPE);
+  MOE_REQUIRE(G == 0 || R == 0 || C == 0 || G * (R / 128) * (C / 128) < (1ll << 31),
+              MOE_ERR_SHAPE);
+  if (G == 0 || R == 0 || C == 0) return MOE_OK;
+  MOE_CHECK_PTR(w);
+  MOE_CHECK_PTR(q);
+  MOE_CHECK_PTR(scale);
+  const DeviceInfo *di = nullptr;
+  const int rc = device_info(&di);
+  if (rc != MOE_OK) return rc;
+  return to_status(launch_quantize_fp8(w, G, R, C, q, scale, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_expert_ffn_fp8(const moe_dims *dims, const moe_bf16 *x_perm, const int32_t *offsets,
+                       const float *perm_gate, const uint8_t *q_g, const float *s_g,
+                       const uint8_t *q_u, const float *s_u, const uint8_t *q_d,
+                       const float *s_d, moe_bf16 *h, moe_bf16 *y_perm, void *ws,
+                       size_t ws_bytes, void *stream) {
+  MOE_REQUIRE(dims != nullptr, MOE_ERR_ARG);
+  MOE_REQUIRE(dims_ok(dims) && fp8_dims_ok(*dims), MOE_ERR_SHAPE);
+  MOE_CHECK_TOKEN_PTR(x_perm, dims->T);
+  MOE_CHECK_PTR(offsets);
+  MOE_CHECK_TOKEN_PTR(perm_gate, dims->T);
+  const Fp8Weights fw{q_g, q_u, q_d, s_g, s_u, s_d};
+  MOE_CHECK_PTR(q_g);
+  MOE_CHECK_PTR(q_u);
+  MOE_CHECK_PTR(q_d);
+  MOE_CHECK_PTR(s_g);
+  MOE_CHECK_PTR(s_u);
+  MOE_CHECK_PTR(s_d);
+  MOE_CHECK_TOKEN_PTR(h, dims->T);
+  MOE_CHECK_TOKEN_PTR(y_perm, dims->T);
+  const Layout L = layout_of(*dims);
+  int rc = check_ws(ws, ws_bytes, L.scratch_end);
+  if (rc != MOE_OK) return rc;
+  const DeviceInfo *di = nullptr;
+  rc = device_info(&di);
+  if (rc != MOE_OK) return rc;
+  return do_expert_ffn(*dims, *di, L, x_perm, offsets, perm_gate, nullptr, nullptr, nullptr, h,
+                       y_perm, ws, static_cast<cudaStream_t>(stream), nullptr, nullptr, nullptr,
+                       &fw);
+}
+
+int moe_forward_fp8(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *W_r,
+                    const float *b, const uint8_t *q_g, const float *s_g, const uint8_t *q_u,
+                    const float *s_u, const uint8_t *q_d, const float *s_d, moe_bf16 *y,
+                    int32_t *counts, void *ws, size_t ws_bytes, void *const *stage_events,
+                    void *stream) {
+  const Fp8Weights fw{q_g, q_u, q_d, s_g, s_u, s_d};
+  return forward_impl(dims, x, W_r, b, nullptr, nullptr, nullptr, y, counts, ws, ws_bytes,
+                      stage_events, stream, &fw);
 }
 
 int moe_last_device_error(void *ws, void *stream) {

@@ -109,6 +109,48 @@ def test_expert_ffn_matches_oracle(name):
     assert st.device_status() == 0
 
 
+@pytest.mark.parametrize("name,T", [("tiny", None), ("mid", 256), ("mid", 333)])
+def test_expert_ffn_gather_matches_oracle_and_unfused(name, T):
+    # The up-projection gathering token rows from x by perm_tok (no x_perm): against the
+    # oracle's expert rows, and bit for bit against moe_expert_ffn on the gathered copy.
+    w = WORKLOADS[name]
+    w, x, wt = _case(w, T=T)
+    ref = oracle.router(x, wt["W_r"], wt["b"], w.K)
+    dsp = oracle.dispatch(ref["topk_idx"], w.N, w.E)
+    rows, gates = _oracle_expert_rows(w, x, wt, ref["topk_idx"], ref["topk_gate"], dsp)
+    A = len(dsp["perm_tok"])
+    st = Stages(w, x, wt)
+    st.x_perm[:A].copy_(x[torch.from_numpy(dsp["perm_tok"]).long()])
+    st.perm_tok[:A].copy_(torch.from_numpy(dsp["perm_tok"]))
+    st.offsets.copy_(torch.from_numpy(dsp["offsets"]))
+    st.perm_gate[:A].copy_(torch.from_numpy(gates.astype(np.float32)))
+    st.expert_ffn()
+    h_ref, y_ref = st.h[:A].clone(), st.y_perm[:A].clone()
+    st.h.zero_()
+    st.y_perm.zero_()
+    mb.moe_expert_ffn_gather(st.dm, st.x, st.perm_tok, st.offsets, st.perm_gate, st.wt["W_g"],
+                             st.wt["W_u"], st.wt["W_d"], st.h, st.y_perm, st.ws)
+    torch.cuda.synchronize()
+    assert st.device_status() == 0
+    assert torch.equal(st.h[:A], h_ref) and torch.equal(st.y_perm[:A], y_ref)
+    assert_y_close(oracle.bf16_to_f64(to_np(st.y_perm)[:A]), rows, f"{name} gathered y_perm")
+
+
+def test_dispatch_without_gather_leaves_x_perm_alone():
+    w, x, wt = _case(WORKLOADS["tiny"])
+    st = Stages(w, x, wt)
+    st.route()
+    st.dispatch()
+    tables = [t.clone() for t in (st.counts, st.offsets, st.perm_tok, st.perm_gate, st.slot_pos)]
+    st.x_perm.fill_(3.0)
+    mb.moe_dispatch(st.dm, st.x, st.topk_idx, st.topk_gate, st.counts, st.offsets, st.perm_tok,
+                    st.perm_gate, st.slot_pos, None, st.ws)
+    torch.cuda.synchronize()
+    for a, b in zip(tables, (st.counts, st.offsets, st.perm_tok, st.perm_gate, st.slot_pos)):
+        assert torch.equal(a, b)
+    assert (st.x_perm == 3.0).all()
+
+
 @pytest.mark.parametrize("name", ["tiny", "mid"])
 def test_combine_matches_oracle(name):
     w = WORKLOADS[name]

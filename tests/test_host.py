@@ -88,6 +88,23 @@ def test_argument_errors_are_reported_before_any_device_work():
     assert lib.moe_last_device_error(None, None) == 1
 
 
+def test_fp8_shape_errors_before_device_work():
+    lib = mb.lib()
+    # R or C not a multiple of 128
+    assert lib.moe_quantize_fp8(P(0x10000), 1, 100, 128, P(0x20000), P(0x30000), None) == 2
+    assert lib.moe_quantize_fp8(P(0x10000), 1, 128, 192, P(0x20000), P(0x30000), None) == 2
+    assert lib.moe_quantize_fp8(None, 0, 128, 128, None, None, None) == 0  # nothing to do
+    # d = 192 is a valid bf16 width but not a whole number of 128-wide scale blocks
+    dm = mb.dims(64, 192, 8, 4, 3, 256)
+    args = [P(0x10000 * (i + 1)) for i in range(10)]  # x, W_r, b, 6 FP8 tensors, y
+    assert lib.moe_forward_fp8(ctypes.byref(dm), *args, None, P(0x1000000),
+                               mb.workspace_size(dm), None, None) == 2
+    dm2 = mb.dims(64, 128, 8, 4, 3, 256)
+    args[3] = P(0)  # NULL codes
+    assert lib.moe_forward_fp8(ctypes.byref(dm2), *args, None, P(0x1000000),
+                               mb.workspace_size(dm2), None, None) == 1
+
+
 def test_variant_switches_are_validated():
     lib = mb.lib()
     dm = mb.dims(64, 128, 8, 4, 3, 256, flags=mb.RENORMALIZE_GATES)
