@@ -44,10 +44,11 @@ LAUNCHES_PER_STEP = 10  # router GEMM, top-K, histogram, scan, permute, gather, 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM traffic per launch of the dominant kernel from an ncu capture (profiles/), valid only
-# while the kernel source is unchanged (sha1 of the GEMM source at capture time).
+# while the kernel and its launch set-up are unchanged (sha1 of the GEMM kernel source and of
+# the file that builds its tensor maps, at capture time).
 NCU_TRAFFIC = {
-    ("prefill", "ffn_up_gemm"): {"bytes_per_launch": 41_834_767_616, "src": "44b67aaf0a11"},
-    ("decode", "ffn_up_gemm"): {"bytes_per_launch": 7_316_203_008, "src": "44b67aaf0a11"},
+    ("prefill", "ffn_up_gemm"): {"bytes_per_launch": 37_801_926_400, "src": "62105494cf85"},
+    ("decode", "ffn_up_gemm"): {"bytes_per_launch": 7_315_725_824, "src": "62105494cf85"},
 }
 
 
@@ -66,7 +67,7 @@ def peaks():
 
 def gemm_source_hash():
     h = hashlib.sha1()
-    for name in ("gemm.cu", "device.cuh", "kernels.cuh"):
+    for name in ("gemm.cu", "device.cuh", "kernels.cuh", "moe_api.cu"):
         with open(os.path.join(ROOT, "mixture_experts_layer_38_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:12]

@@ -72,8 +72,12 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // Row-major bf16 matrix [rows, cols] read in boxes of 64 columns x box_rows rows, 128-byte
 // swizzle (the layout the tcgen05 descriptors expect), zero fill outside the matrix.
+// L2 promotion: each box row is a 128-byte segment; promoting misses to 256 bytes fetches the
+// next k-slice early, which helps weight streaming (128-token tiles: decode 8% faster) but at
+// 256-token tiles the promoted halves are often evicted before use and fetched again (prefill
+// DRAM traffic 10% higher), so those launches promote to 128 bytes.
 bool make_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
-              uint32_t box_rows) {
+              uint32_t box_rows, bool promote256 = true) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {cols, rows};
@@ -82,7 +86,8 @@ bool make_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
   cuuint32_t estride[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
             box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+            promote256 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
 }
 
@@ -108,10 +113,11 @@ struct Fp8Weights {
   const float *s_g, *s_u, *s_d;
 };
 
-bool make_act_maps(GemmArgs &a, const void *base, uint64_t rows, uint64_t cols) {
+bool make_act_maps(GemmArgs &a, const void *base, uint64_t rows, uint64_t cols,
+                   bool promote256 = true) {
   for (int i = 0; i < 4; ++i)
-    if (!make_map(&a.map_b[i], base, rows, cols, 128u >> i)) return false;
-  return make_map(&a.map_b256, base, rows, cols, 256);
+    if (!make_map(&a.map_b[i], base, rows, cols, 128u >> i, promote256)) return false;
+  return make_map(&a.map_b256, base, rows, cols, 256, promote256);
 }
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -229,10 +235,12 @@ int do_route(const moe_dims &d, const DeviceInfo &di, const Layout &L, const moe
   int *status = at<int>(ws, L.status);
   float *logits = at<float>(ws, L.logits);
   GemmArgs a{};
-  if (!make_map(&a.map_a0, W_r, (uint64_t)E, (uint64_t)d.d, 128) ||
-      !make_map(&a.map_a1, W_r, (uint64_t)E, (uint64_t)d.d, 128) ||
-      !make_map(&a.map_a01, W_r, (uint64_t)E, (uint64_t)d.d, 256) ||
-      !make_act_maps(a, x, (uint64_t)d.T, (uint64_t)d.d)) {
+  const int router_tile = gemm_tile_tokens(d.T, 1, d.d);
+  const bool p256 = router_tile != 256;
+  if (!make_map(&a.map_a0, W_r, (uint64_t)E, (uint64_t)d.d, 128, p256) ||
+      !make_map(&a.map_a1, W_r, (uint64_t)E, (uint64_t)d.d, 128, p256) ||
+      !make_map(&a.map_a01, W_r, (uint64_t)E, (uint64_t)d.d, 256, p256) ||
+      !make_act_maps(a, x, (uint64_t)d.T, (uint64_t)d.d, p256)) {
     return MOE_ERR_CUDA;
   }
   a.group_offsets = nullptr;
@@ -248,7 +256,7 @@ int do_route(const moe_dims &d, const DeviceInfo &di, const Layout &L, const moe
   a.status = status;
   const long long tiles = (long long)((d.T + 127) / 128) * ((E + 255) / 256) * L.splits;
   const int grid = (int)(tiles < di.sms ? tiles : di.sms);
-  cudaError_t e = launch_grouped_gemm(kEpiF32, a, grid, gemm_tile_tokens(d.T, 1, d.d), stream);
+  cudaError_t e = launch_grouped_gemm(kEpiF32, a, grid, router_tile, stream);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if (record(events, 1, stream) != MOE_OK) return MOE_ERR_CUDA;
   return to_status(
@@ -283,15 +291,18 @@ int do_expert_ffn(const moe_dims &d, const DeviceInfo &di, const Layout &L,
   GemmArgs up{};
   // Token rows: the grouped copy x_perm, or (perm_tok given) gathered from x by the GEMM.
   const bool gather = perm_tok != nullptr;
+  const int tile_tokens = gemm_tile_tokens((long long)rows, d.N, d.d);
+  const bool p256 = fw != nullptr || tile_tokens != 256;  // L2 promotion, see make_map
   const bool ok_w = fw != nullptr
       ? make_map_u8(&up.map_a0, fw->q_g, (uint64_t)d.N * d.I, (uint64_t)d.d) &&
             make_map_u8(&up.map_a1, fw->q_u, (uint64_t)d.N * d.I, (uint64_t)d.d) &&
             make_map_u8(&up.map_a01, fw->q_g, (uint64_t)d.N * d.I, (uint64_t)d.d)
-      : make_map(&up.map_a0, W_g, (uint64_t)d.N * d.I, (uint64_t)d.d, 128) &&
-            make_map(&up.map_a1, W_u, (uint64_t)d.N * d.I, (uint64_t)d.d, 128) &&
-            make_map(&up.map_a01, W_g, (uint64_t)d.N * d.I, (uint64_t)d.d, 256);
+      : make_map(&up.map_a0, W_g, (uint64_t)d.N * d.I, (uint64_t)d.d, 128, p256) &&
+            make_map(&up.map_a1, W_u, (uint64_t)d.N * d.I, (uint64_t)d.d, 128, p256) &&
+            make_map(&up.map_a01, W_g, (uint64_t)d.N * d.I, (uint64_t)d.d, 256, p256);
   if (!ok_w ||
-      !make_act_maps(up, gather ? x : x_perm, gather ? (uint64_t)d.T : rows, (uint64_t)d.d) ||
+      !make_act_maps(up, gather ? x : x_perm, gather ? (uint64_t)d.T : rows, (uint64_t)d.d,
+                     p256) ||
       (gather && !make_map(&up.map_bg, x, (uint64_t)d.T, (uint64_t)d.d, 1))) {
     return MOE_ERR_CUDA;
   }
@@ -312,7 +323,6 @@ int do_expert_ffn(const moe_dims &d, const DeviceInfo &di, const Layout &L,
     up.scale_a1 = fw->s_u;
     up.scale_ld = d.d / 128;
   }
-  const int tile_tokens = gemm_tile_tokens((long long)rows, d.N, d.d);
   if ((fw != nullptr ? launch_grouped_gemm_fp8(kEpiSwiGLU, up, di.sms, stream)
                      : launch_grouped_gemm(kEpiSwiGLU, up, di.sms, tile_tokens, stream)) !=
       cudaSuccess)
@@ -324,10 +334,10 @@ int do_expert_ffn(const moe_dims &d, const DeviceInfo &di, const Layout &L,
       ? make_map_u8(&down.map_a0, fw->q_d, (uint64_t)d.N * d.d, (uint64_t)d.I) &&
             make_map_u8(&down.map_a1, fw->q_d, (uint64_t)d.N * d.d, (uint64_t)d.I) &&
             make_map_u8(&down.map_a01, fw->q_d, (uint64_t)d.N * d.d, (uint64_t)d.I)
-      : make_map(&down.map_a0, W_d, (uint64_t)d.N * d.d, (uint64_t)d.I, 128) &&
-            make_map(&down.map_a1, W_d, (uint64_t)d.N * d.d, (uint64_t)d.I, 128) &&
-            make_map(&down.map_a01, W_d, (uint64_t)d.N * d.d, (uint64_t)d.I, 256);
-  if (!ok_wd || !make_act_maps(down, h, rows, (uint64_t)d.I)) {
+      : make_map(&down.map_a0, W_d, (uint64_t)d.N * d.d, (uint64_t)d.I, 128, p256) &&
+            make_map(&down.map_a1, W_d, (uint64_t)d.N * d.d, (uint64_t)d.I, 128, p256) &&
+            make_map(&down.map_a01, W_d, (uint64_t)d.N * d.d, (uint64_t)d.I, 256, p256);
+  if (!ok_wd || !make_act_maps(down, h, rows, (uint64_t)d.I, p256)) {
     return MOE_ERR_CUDA;
   }
   down.group_offsets = offsets;

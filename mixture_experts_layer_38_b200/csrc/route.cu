@@ -1,4 +1,5 @@
-// route.cu -- softmax router R and biased top-K selection, one thread block per token.
+// route.cu -- softmax router R and biased top-K selection: one thread block per token, or one
+// warp per token for pools of up to 256 experts.
 //
 // "衝上熱搜！美團大模型，靠「快」火了", §零計算專家: R is a softmax router over the N FFN experts
 // and Z zero-computation experts; a per-expert bias b_i adjusts the routing score used to pick
@@ -23,7 +24,7 @@ namespace {
 // Selection key of expert id with score s:
 // (order-preserving bits of s) << 32 | (0xffffffff - id)  ->  larger score, then lower id.
 constexpr int kBlockThreads = 256;
-constexpr int kPerThread = 4;  // E <= 1024
+constexpr int kMaxPerThread = 4;  // E <= 1024
 
 __device__ __forceinline__ uint64_t score_key(float s, int id) {
   uint32_t u = __float_as_uint(s);
@@ -55,7 +56,10 @@ __device__ __forceinline__ float block_reduce(float v, bool is_max, float *red) 
   return r;
 }
 
-__global__ void __launch_bounds__(kBlockThreads)
+// kPerThread experts per thread (E <= 256 * kPerThread).  With three, at most 64 registers so
+// that four blocks share an SM.
+template <int kPerThread>
+__global__ void __launch_bounds__(kBlockThreads, kPerThread <= 3 ? 4 : 3)
     route_topk_block_kernel(const float *__restrict__ logits, int splits, int T, int E, int ld,
                             int K, const float *__restrict__ b, bool renormalize,
                             int32_t *__restrict__ topk_idx, float *__restrict__ topk_gate,
@@ -156,6 +160,102 @@ __global__ void __launch_bounds__(kBlockThreads)
   }
 }
 
+// Pools of up to 256 experts: one warp per token (8 tokens per block), lane i holding experts
+// i, i + 32, ...; the same keys and K+1 argmax rounds as above, with warp shuffles only, so a
+// small pool does not leave most of a 256-thread block idle.
+constexpr int kWarpPer = 8;  // experts per lane: E <= 256
+
+__global__ void __launch_bounds__(256)
+    route_topk_warp_kernel(const float *__restrict__ logits, int splits, int T, int E, int ld,
+                           int K, const float *__restrict__ b, bool renormalize,
+                           int32_t *__restrict__ topk_idx, float *__restrict__ topk_gate,
+                           float *__restrict__ gap, int *status) {
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const int lane = threadIdx.x & 31;
+  const long long split_stride = (long long)T * ld;
+  float p[kWarpPer];
+  float m = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < kWarpPer; ++j) {
+    const int e = lane + 32 * j;
+    float v = -INFINITY;
+    if (e < E) {
+      const float *src = logits + (long long)t * ld + e;
+      v = src[0];
+      for (int sp = 1; sp < splits; ++sp) v += src[sp * split_stride];
+    }
+    p[j] = v;
+    m = fmaxf(m, v);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  float z = 0.f;
+#pragma unroll
+  for (int j = 0; j < kWarpPer; ++j) {
+    p[j] = (lane + 32 * j < E) ? expf(p[j] - m) : 0.f;
+    z += p[j];
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+  uint64_t key[kWarpPer];
+#pragma unroll
+  for (int j = 0; j < kWarpPer; ++j) {
+    const int e = lane + 32 * j;
+    p[j] = __fdiv_rn(p[j], z);
+    key[j] = (e < E) ? score_key(__fadd_rn(p[j], __ldg(b + e)), e) : 0ull;
+  }
+  const int rounds = K < E ? K + 1 : K;
+  int my_id = 0x7fffffff;  // lane k keeps the k-th selected expert
+  float my_p = 0.f, s_k1 = 0.f, s_k = 0.f;
+  for (int k = 0; k < rounds; ++k) {
+    uint64_t best = key[0];
+#pragma unroll
+    for (int j = 1; j < kWarpPer; ++j) best = key[j] > best ? key[j] : best;
+    best = warp_max_u64(best);
+    if (best == 0ull) {  // nothing left that is selectable (non-finite scores): flag, skip
+      if (lane == 0) record_status(status, MOE_DEV_BAD_EXPERT);
+      continue;
+    }
+    const int id = (int)(0xffffffffu - (uint32_t)(best & 0xffffffffu));
+    const int owner = id & 31, jo = id >> 5;
+    float pv = 0.f;
+#pragma unroll
+    for (int j = 0; j < kWarpPer; ++j) {
+      if (j == jo && lane == owner) {
+        pv = p[j];
+        key[j] = 0ull;
+      }
+    }
+    pv = __shfl_sync(0xffffffffu, pv, owner);
+    const float sv = __fadd_rn(pv, __ldg(b + id));
+    if (lane == k) {
+      my_id = id;
+      my_p = pv;
+    }
+    if (k == K - 1) s_k1 = sv;
+    if (k == K) s_k = sv;
+  }
+  int rank = 0;
+  for (int k2 = 0; k2 < K; ++k2) {
+    const int other = __shfl_sync(0xffffffffu, my_id, k2);
+    rank += other < my_id;
+  }
+  float g = lane < K ? my_p : 0.f;
+  if (renormalize) {
+    float sum = g;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+      sum = __fadd_rn(sum, __shfl_xor_sync(0xffffffffu, sum, off));
+    g = __fdiv_rn(g, sum);
+  }
+  if (lane < K) {
+    topk_idx[(long long)t * K + rank] = my_id;
+    topk_gate[(long long)t * K + rank] = g;
+  }
+  if (gap != nullptr && lane == 0) gap[t] = (K < E) ? __fsub_rn(s_k1, s_k) : INFINITY;
+}
+
 }  // namespace
 
 cudaError_t launch_route_topk(const float *logits, int splits, int T, int E, int K,
@@ -163,8 +263,15 @@ cudaError_t launch_route_topk(const float *logits, int splits, int T, int E, int
                               float *topk_gate, float *gap, int *status, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
   const int ld = (E + 3) & ~3;
-  route_topk_block_kernel<<<T, kBlockThreads, 0, stream>>>(
-      logits, splits, T, E, ld, K, b, renormalize, topk_idx, topk_gate, gap, status);
+  if (E <= 32 * kWarpPer)
+    route_topk_warp_kernel<<<(T + 7) / 8, 256, 0, stream>>>(
+        logits, splits, T, E, ld, K, b, renormalize, topk_idx, topk_gate, gap, status);
+  else if (E <= 3 * kBlockThreads)
+    route_topk_block_kernel<3><<<T, kBlockThreads, 0, stream>>>(
+        logits, splits, T, E, ld, K, b, renormalize, topk_idx, topk_gate, gap, status);
+  else
+    route_topk_block_kernel<kMaxPerThread><<<T, kBlockThreads, 0, stream>>>(
+        logits, splits, T, E, ld, K, b, renormalize, topk_idx, topk_gate, gap, status);
   return cudaGetLastError();
 }
 

@@ -106,3 +106,44 @@ def test_skewed_pid_full_size(big_weights):
     assert means[0] > w.pid_target + 1.0  # the Zipf offset favours FFN experts at the start
     assert abs(means[-10:].mean() - w.pid_target) < 0.15
     assert (b[w.N:] == wt["b"][w.N:]).all()  # zero-expert biases never move
+
+
+def test_decode_fp8_full_size(big_weights):
+    # Block-wise FP8 expert weights at full size, in the launch configuration the benchmark's
+    # --fp8 leg times (moe_forward_fp8): sampled tokens against the oracle run on the
+    # dequantised weights (q * 2^e, exact in bf16).
+    w = WORKLOADS["decode"]
+    x = make_tokens(w, DEV, seed=0)
+    dm = mb.dims(w.T, w.d, w.N, w.Z, w.K, w.I)
+    fw = mb.quantize_expert_weights_fp8(dm, big_weights["W_g"], big_weights["W_u"],
+                                        big_weights["W_d"])
+    ws = mb.alloc_workspace(dm, DEV)
+    y = torch.empty((w.T, w.d), dtype=torch.bfloat16, device=DEV)
+    counts = torch.zeros(w.E, dtype=torch.int32, device=DEV)
+    mb.moe_forward_fp8(dm, x, big_weights["W_r"], big_weights["b"], fw, y, counts, ws)
+    torch.cuda.synchronize()
+    assert mb.moe_last_device_error(ws) == 0
+    assert int(counts.sum().item()) == w.T * w.K
+
+    def fetch_deq(e):
+        out = []
+        for k in ("g", "u", "d"):
+            bits = oracle.dequantize_fp8_blocks(fw["q_" + k][e:e + 1].cpu().numpy(),
+                                                fw["s_" + k][e:e + 1].cpu().numpy())[0]
+            out.append(bits)
+        return tuple(out)
+    n_sample = 24
+    tokens = np.sort(np.random.default_rng(5).choice(w.T, n_sample, replace=False))
+    xs = x[torch.from_numpy(tokens).to(DEV)].cpu()
+    W_r, b = big_weights["W_r"].cpu(), big_weights["b"].cpu()
+    ref = oracle.router(xs, W_r, b, w.K, want_scores=True)
+    out = oracle.forward_sampled(np.arange(n_sample), xs, W_r, b, w.N, w.Z, w.K, fetch_deq,
+                                 routing=ref)
+    st = Stages(w, x, big_weights)
+    st.route()
+    idx = to_np(st.topk_idx)[tokens]
+    check_routing(idx, to_np(st.topk_gate)[tokens], ref, ref["scores"])
+    same = (idx == ref["topk_idx"]).all(axis=1)
+    y_s = oracle.bf16_to_f64(to_np(y))[tokens]
+    assert_y_close(y_s[same], out["y"][same], "decode fp8 y")
+    del fw
