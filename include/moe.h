@@ -167,10 +167,10 @@ int moe_expert_ffn(const moe_dims *dims, const moe_bf16 *x_perm, const int32_t *
                    size_t ws_bytes, void *stream);
 
 /* moe_expert_ffn with the dispatch gather fused into the up-projection: grouped row r's
- * token row is read straight from x[perm_tok[r]] by the GEMM's loads (TMA row gathers), so no
- * x_perm copy is written or read: T*K*d*2 bytes of memory saved, at a cost in speed (the
- * row-by-row loads limit the up-projection; moe_forward keeps the copy).  Arguments as
- * moe_expert_ffn, with
+ * token row is read straight from x[perm_tok[r]] by the GEMM's own loads, so no x_perm copy is
+ * written or read: T*K*d*2 bytes of memory saved, at some cost in speed at large T (the
+ * row-by-row copies; moe_forward keeps the copy).  A perm_tok value outside [0, T) is
+ * reported as MOE_DEV_BAD_ROWS and row 0 is read instead.  Arguments as moe_expert_ffn, with
  *   x        [T, d] bf16      the tokens (as given to moe_dispatch)
  *   perm_tok [T*K] int32      token of each grouped row, from moe_dispatch (values in [0, T))
  * in place of x_perm.  h and y_perm are bit-identical to moe_expert_ffn on the gathered

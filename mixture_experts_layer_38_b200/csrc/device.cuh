@@ -85,18 +85,18 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *m
       : "memory");
 }
 
-// Row-gather bulk copy (sm_100a): four rows r0..r3 of a 2-D tensor map whose box is 64
-// columns x 1 row, columns [c0, c0 + 64), land in shared memory as 4 consecutive 128-byte rows
-// (swizzled by destination address like a tiled load); completes 512 bytes on `bar`.
-__device__ __forceinline__ void tma_gather4(void *smem_dst, const CUtensorMap *map,
-                                            uint64_t *bar, int c0, int r0, int r1, int r2,
-                                            int r3, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1),
-      "r"(r2), "r"(r3), "l"(policy)
-      : "memory");
+// 16-byte asynchronous copy global -> shared, cached in L2 only.
+__device__ __forceinline__ void cp_async_16(void *smem_dst, const void *gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)),
+               "l"(gmem_src)
+               : "memory");
+}
+
+// One arrival on `bar` once all of this thread's earlier cp.async copies have landed (the
+// barrier's expected count includes it: .noinc).
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t *bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
 }
 
 // Orders this thread's generic-proxy shared-memory stores before later async-proxy reads

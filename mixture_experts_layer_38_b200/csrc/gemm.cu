@@ -70,8 +70,13 @@ constexpr int kSmemPrefix = 2 * (kMaxGroups + 4) * 4;  // full-tile and tail-til
 // codes and the MMA its token rows; a slot once the MMA has read it.
 constexpr int kQTile = kBM * kBK;            // 8 KB of E4M3 codes per weight block
 constexpr int kConvWarps = 8;
+// Row gather (GA): four loader warps copy the token rows of each stage from x[row_index[r]]
+// with 16-byte cp.async into the swizzled token tile; the stage barrier expects one arrival
+// per loader thread besides the producer's.
+constexpr int kLoadWarps = 4;
+constexpr int kLoadThreads = 32 * kLoadWarps;
 
-template <int BN, bool WQ = false>
+template <int BN, bool WQ = false, bool GA = false>
 struct Cfg {
   static constexpr int kAccBufs = BN <= 128 ? 2 : 1;
   static constexpr int kStage = (WQ ? 2 * kQTile : 2 * kTileA) + BN * kBK * 2;
@@ -79,7 +84,8 @@ struct Cfg {
   static constexpr int kCRing = kCSlots * 2 * kTileA;
   static constexpr int kStages = (192 * 1024 - kCRing) / kStage;
   static constexpr int kNumBars = 2 * kStages + 2 * kAccBufs + 1 + 2 * kCSlots;
-  static constexpr int kThreads = 64 + 32 * kEpiWarps + (WQ ? 32 * kConvWarps : 0);
+  static constexpr int kThreads =
+      64 + 32 * kEpiWarps + (WQ ? 32 * kConvWarps : 0) + (GA ? kLoadThreads : 0);
   static constexpr int kSmemBytes = 1024 + kStages * kStage + kCRing + kSmemStaging +
                                     kSmemPrefix + kNumBars * 8 + 16;
   static_assert(kAccBufs * 2 * BN <= kTmemCols, "TMEM holds 512 columns");
@@ -377,9 +383,9 @@ __device__ __forceinline__ void convert_fp8_block(const uint8_t *q, uint8_t *dst
 }
 
 template <int EPI, int BN, bool WQ, bool GATHER>
-__global__ void __launch_bounds__(Cfg<BN, WQ>::kThreads, 1)
+__global__ void __launch_bounds__(Cfg<BN, WQ, GATHER>::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ GemmArgs args) {
-  using C = Cfg<BN, WQ>;
+  using C = Cfg<BN, WQ, GATHER>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -405,7 +411,7 @@ __global__ void __launch_bounds__(Cfg<BN, WQ>::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&full_bar[s], 1);
+      mbar_init(&full_bar[s], GATHER ? 1 + kLoadThreads : 1);
       mbar_init(&empty_bar[s], WQ ? 1 + kConvWarps : 1);  // WQ: the converters read it too
     }
     for (int b = 0; b < C::kAccBufs; ++b) {
@@ -427,7 +433,6 @@ __global__ void __launch_bounds__(Cfg<BN, WQ>::kThreads, 1)
     tma_prefetch_desc(&args.map_b256);
 #pragma unroll
     for (int i = 0; i < 4; ++i) tma_prefetch_desc(&args.map_b[i]);
-    if (GATHER) tma_prefetch_desc(&args.map_bg);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -445,11 +450,9 @@ __global__ void __launch_bounds__(Cfg<BN, WQ>::kThreads, 1)
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
-    // Lane 0 issues the weight loads and the tiled token loads.  In gather mode the whole warp
-    // runs the loop and every lane issues tile::gather4 loads of 4 token rows each (groups
-    // `lane` and `lane + 32` of the tile's nb rows) after lane 0 has armed the stage's barrier.
-    constexpr bool gather = GATHER;
-    if (gather || lane == 0) {
+    // Lane 0 issues the weight loads and the tiled token loads (in gather mode the loader warps
+    // fetch the token rows instead).
+    if (lane == 0) {
       // Weights of a group with a single token tile are read once: stream them past L2
       // (evict-first) so they do not push out the tiles other CTAs are still re-reading.
       const uint64_t pol_w_reused = l2_policy_evict_normal();
@@ -461,21 +464,12 @@ __global__ void __launch_bounds__(Cfg<BN, WQ>::kThreads, 1)
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < sched.total; tile += gridDim.x) {
         const Tile t = decode_tile<EPI, BN>(args, sched, tile);
-        const uint32_t bytes = (WQ ? kQTile : kTileA) * (t.has_a1 ? 2 : 1) + t.nb * kBK * 2;
+        const uint32_t bytes = (WQ ? kQTile : kTileA) * (t.has_a1 ? 2 : 1) +
+                               (GATHER ? 0 : t.nb * kBK * 2);
         const uint64_t pol_w = t.once ? pol_w_once : pol_w_reused;
-        int rix[8];  // gather mode: source rows of this lane's two 4-row groups
-        if (gather) {
-  #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int r = (i < 4 ? lane : lane + 32) * 4 + (i & 3);
-            rix[i] = __ldg(args.row_index + t.row0 + min(r, t.n_valid - 1));  // pad: a valid row
-          }
-        }
-        const int groups = t.nb >> 2;
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
-          if (!(gather ? warp_wait(&empty_bar[stage], phase ^ 1, abort_flag)
-                       : mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag))) {
-            if (lane == 0) signal_abort(args, abort_flag);
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag)) {
+            signal_abort(args, abort_flag);
             ok = false;
             break;
           }
@@ -483,54 +477,43 @@ __global__ void __launch_bounds__(Cfg<BN, WQ>::kThreads, 1)
           uint8_t *sa1 = sa0 + kTileA;
           uint8_t *sb = sa0 + (WQ ? 2 * kQTile : 2 * kTileA);
           const int kc = kb * kBK;
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&full_bar[stage], bytes);
-            if (WQ) {  // E4M3 codes of both weight blocks at the start of the stage
-              tma_load_2d(sa0, &args.map_a0, &full_bar[stage], kc, t.a0_row, pol_w);
-              if (t.has_a1)
-                tma_load_2d(sa0 + kQTile, &args.map_a1, &full_bar[stage], kc, t.a1_row, pol_w);
-            } else if (kWideBoxes && EPI != kEpiSwiGLU && t.has_a1) {
-              tma_load_2d(sa0, &args.map_a01, &full_bar[stage], kc, t.a0_row, pol_w);
-            } else {
-              tma_load_2d(sa0, &args.map_a0, &full_bar[stage], kc, t.a0_row, pol_w);
-              if (t.has_a1)
-                tma_load_2d(sa1, &args.map_a1, &full_bar[stage], kc, t.a1_row, pol_w);
-            }
-            if (!gather) {
-              // Token rows in boxes of 256 / 128 (as many as needed), then 64 / 32 / 16.
-              int r = 0;
-              if (kWideBoxes && t.nb == 256) {
-                tma_load_2d(sb, &args.map_b256, &full_bar[stage], kc, t.row0, pol_x);
-                r = 256;
-              }
-              for (; t.nb - r >= 128; r += 128)
-                tma_load_2d(sb + r * (kBK * 2), &args.map_b[0], &full_bar[stage], kc,
-                            t.row0 + r, pol_x);
-#pragma unroll
-              for (int i = 1; i < 4; ++i) {
-                const int box = 128 >> i;
-                if (t.nb - r >= box) {
-                  tma_load_2d(sb + r * (kBK * 2), &args.map_b[i], &full_bar[stage], kc,
-                              t.row0 + r, pol_x);
-                  r += box;
-                }
-              }
-            }
+          mbar_arrive_expect_tx(&full_bar[stage], bytes);
+          if (WQ) {  // E4M3 codes of both weight blocks at the start of the stage
+            tma_load_2d(sa0, &args.map_a0, &full_bar[stage], kc, t.a0_row, pol_w);
+            if (t.has_a1)
+              tma_load_2d(sa0 + kQTile, &args.map_a1, &full_bar[stage], kc, t.a1_row, pol_w);
+          } else if (kWideBoxes && EPI != kEpiSwiGLU && t.has_a1) {
+            tma_load_2d(sa0, &args.map_a01, &full_bar[stage], kc, t.a0_row, pol_w);
+          } else {
+            tma_load_2d(sa0, &args.map_a0, &full_bar[stage], kc, t.a0_row, pol_w);
+            if (t.has_a1)
+              tma_load_2d(sa1, &args.map_a1, &full_bar[stage], kc, t.a1_row, pol_w);
           }
-          if (gather) {
-            __syncwarp();  // the barrier is armed before any gathered bytes can land
-            if (lane < groups)
-              tma_gather4(sb + lane * (4 * kBK * 2), &args.map_bg, &full_bar[stage], kc, rix[0],
-                          rix[1], rix[2], rix[3], pol_x);
-            if (lane + 32 < groups)
-              tma_gather4(sb + (lane + 32) * (4 * kBK * 2), &args.map_bg, &full_bar[stage], kc,
-                          rix[4], rix[5], rix[6], rix[7], pol_x);
+          if (!GATHER) {
+            // Token rows in boxes of 256 / 128 (as many as needed), then 64 / 32 / 16.
+            int r = 0;
+            if (kWideBoxes && t.nb == 256) {
+              tma_load_2d(sb, &args.map_b256, &full_bar[stage], kc, t.row0, pol_x);
+              r = 256;
+            }
+            for (; t.nb - r >= 128; r += 128)
+              tma_load_2d(sb + r * (kBK * 2), &args.map_b[0], &full_bar[stage], kc, t.row0 + r,
+                          pol_x);
+#pragma unroll
+            for (int i = 1; i < 4; ++i) {
+              const int box = 128 >> i;
+              if (t.nb - r >= box) {
+                tma_load_2d(sb + r * (kBK * 2), &args.map_b[i], &full_bar[stage], kc,
+                            t.row0 + r, pol_x);
+                r += box;
+              }
+            }
           }
           ++issued;
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
         }
       }
-      if (!ok && lane == 0) {
+      if (!ok) {
         // Drain the copies that may still be landing in the ring (bounded).
         for (long long i = 1; i <= issued && i <= C::kStages; ++i) {
           const long long idx = issued - i;
@@ -572,6 +555,9 @@ __global__ void __launch_bounds__(Cfg<BN, WQ>::kThreads, 1)
             break;
           }
           tc_fence_after();
+          // Gathered token rows were written through the generic proxy (cp.async): order them
+          // before the tensor cores' async-proxy reads.
+          if (GATHER) fence_proxy_async_shared();
           const uint32_t sbase = smem_u32(ring + stage * C::kStage);
           const uint32_t abase = WQ ? smem_u32(cring + cslot * (2 * kTileA)) : sbase;
           const uint32_t bbase = sbase + (WQ ? 2 * kQTile : 2 * kTileA);
@@ -598,6 +584,47 @@ __global__ void __launch_bounds__(Cfg<BN, WQ>::kThreads, 1)
         umma_commit(drain_bar);
         const long long t0 = clock64();
         while (!mbar_try_wait(drain_bar, 0) && clock64() - t0 < kDrainLimitCycles) {}
+      }
+    }
+  } else if (GATHER && warp >= 2 + kEpiWarps) {
+    // ---------------------------------------------------------------- row-gather loaders
+    // Thread g copies the 16-byte chunk j = g % 8 of rows g / 8, g / 8 + 16, ... of each
+    // stage's token tile, so every warp moves whole 128-byte row segments; the chunk lands at
+    // its 128-byte-swizzled place (chunk j of row r at (j ^ (r % 8)) * 16).
+    const int g = (int)threadIdx.x - (2 + kEpiWarps) * 32;
+    const int j = g & 7, r0 = g >> 3, sw = r0 & 7;
+    const uint16_t *src = reinterpret_cast<const uint16_t *>(args.gather_src);
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < sched.total; tile += gridDim.x) {
+      const Tile t = decode_tile<EPI, BN>(args, sched, tile);
+      const int nrow = t.nb >> 4;  // rows of this thread: r0 + 16 * i, i < nrow (<= 16)
+      int rix[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        int v = i < nrow ? __ldg(args.row_index + t.row0 + min(r0 + 16 * i, t.n_valid - 1)) : 0;
+        if (v < 0 || v >= args.gather_rows) {  // a bad index: report it, read row 0 instead
+          record_status(args.status, MOE_DEV_BAD_ROWS);
+          v = 0;
+        }
+        rix[i] = v;
+      }
+      for (int kb = t.kb0; kb < t.kb1; ++kb) {
+        if (!warp_wait(&empty_bar[stage], phase ^ 1, abort_flag)) {
+          if (lane == 0) signal_abort(args, abort_flag);
+          ok = false;
+          break;
+        }
+        uint8_t *sb = ring + stage * C::kStage + 2 * kTileA;
+        const uint16_t *col = src + kb * kBK + j * 8;
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          if (i < nrow)
+            cp_async_16(sb + (r0 + 16 * i) * (kBK * 2) + ((j ^ sw) << 4),
+                        col + (long long)rix[i] * args.K);
+        cp_async_mbar_arrive_noinc(&full_bar[stage]);
+        if (++stage == C::kStages) { stage = 0; phase ^= 1; }
       }
     }
   } else if (WQ && warp >= 2 + kEpiWarps) {
@@ -672,7 +699,7 @@ template <int EPI, int BN, bool WQ = false, bool GATHER = false>
 cudaError_t set_smem_limit() {
   return cudaFuncSetAttribute(grouped_gemm_kernel<EPI, BN, WQ, GATHER>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              Cfg<BN, WQ>::kSmemBytes);
+                              Cfg<BN, WQ, GATHER>::kSmemBytes);
 }
 
 template <int BN>
@@ -682,7 +709,8 @@ cudaError_t launch_bn(int epi, const GemmArgs &args, int grid, cudaStream_t stre
   switch (epi) {
     case kEpiSwiGLU:
       if (args.row_index != nullptr)
-        grouped_gemm_kernel<kEpiSwiGLU, BN, false, true><<<grid, threads, smem, stream>>>(args);
+        grouped_gemm_kernel<kEpiSwiGLU, BN, false, true>
+            <<<grid, Cfg<BN, false, true>::kThreads, smem, stream>>>(args);
       else
         grouped_gemm_kernel<kEpiSwiGLU, BN, false, false><<<grid, threads, smem, stream>>>(args);
       break;

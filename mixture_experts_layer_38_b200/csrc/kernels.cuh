@@ -35,10 +35,11 @@ struct GemmArgs {
   const float *row_scale;        // kEpiGated: per-row gate
   int *status;                   // device status word
   // Row gather (up-projection only): when row_index is set, activation row r is row
-  // row_index[r] of the matrix behind map_bg (64 x 1 boxes), fetched with tile::gather4;
+  // row_index[r] of the row-major bf16 matrix gather_src (K columns), copied by loader warps;
   // map_b / map_b256 are then unused.
   const int *row_index;
-  CUtensorMap map_bg;
+  const void *gather_src;
+  int gather_rows;               // rows of gather_src; row indices outside are reported, not read
   // FP8 weights (launch_grouped_gemm_fp8): map_a0 / map_a1 cover E4M3 codes (64 x 128 boxes,
   // no swizzle); the scale of the 128 x 128 block holding weight row r, column k is
   // scale_a0/1[(r / 128) * scale_ld + k / 128].

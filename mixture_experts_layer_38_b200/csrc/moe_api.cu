@@ -302,11 +302,12 @@ int do_expert_ffn(const moe_dims &d, const DeviceInfo &di, const Layout &L,
             make_map(&up.map_a01, W_g, (uint64_t)d.N * d.I, (uint64_t)d.d, 256, p256);
   if (!ok_w ||
       !make_act_maps(up, gather ? x : x_perm, gather ? (uint64_t)d.T : rows, (uint64_t)d.d,
-                     p256) ||
-      (gather && !make_map(&up.map_bg, x, (uint64_t)d.T, (uint64_t)d.d, 1))) {
+                     p256)) {
     return MOE_ERR_CUDA;
   }
   up.row_index = perm_tok;
+  up.gather_src = x;
+  up.gather_rows = d.T;
   up.group_offsets = offsets;
   up.num_groups = d.N;
   up.rows = (int)rows;
@@ -573,8 +574,8 @@ int forward_impl(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *W_r, c
   rc = do_route(d, *di, L, x, W_r, b, topk_idx, topk_gate, at<float>(ws, L.gap), ws, s, ev);
   if (rc != MOE_OK) return rc;
   if ((rc = record(ev, 2, s)) != MOE_OK) return rc;
-  // The gathered copy x_perm and tiled token loads: faster than gathering rows inside the
-  // up-projection (moe_expert_ffn_gather), whose row-by-row loads limit the GEMM.
+  // The gathered copy x_perm and tiled token loads: faster at large T than gathering rows
+  // inside the up-projection (moe_expert_ffn_gather), whose row-by-row copies cost more.
   rc = do_dispatch(d, *di, L, x, topk_idx, topk_gate, cnt, offsets, perm_tok, perm_gate,
                    slot_pos, x_perm, ws, s);
   if (rc != MOE_OK) return rc;

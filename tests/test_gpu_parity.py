@@ -267,6 +267,21 @@ def test_zero_tokens():
     assert st.device_status() == 0
 
 
+def test_zero_tokens_gather_and_fp8_paths():
+    w = Workload("t0", T=0, d=128, N=8, Z=4, K=3, I=256)
+    wt = make_weights(w)
+    x = torch.zeros((0, w.d), dtype=torch.bfloat16)
+    st = Stages(w, x, wt)
+    mb.moe_expert_ffn_gather(st.dm, st.x, st.perm_tok, st.offsets, st.perm_gate, st.wt["W_g"],
+                             st.wt["W_u"], st.wt["W_d"], st.h, st.y_perm, st.ws)
+    fw = mb.quantize_expert_weights_fp8(st.dm, st.wt["W_g"], st.wt["W_u"], st.wt["W_d"])
+    st.counts.fill_(5)
+    mb.moe_forward_fp8(st.dm, st.x, st.wt["W_r"], st.wt["b"], fw, st.y, st.counts, st.ws)
+    torch.cuda.synchronize()
+    assert (st.counts == 0).all()
+    assert st.device_status() == 0
+
+
 @pytest.mark.parametrize("T", [1, 77, 300])
 def test_ragged_token_counts(T):
     w, x, wt = _case(WORKLOADS["tiny"], T=T, seed=T)
