@@ -47,8 +47,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # while the kernel and its launch set-up are unchanged (sha1 of the GEMM kernel source and of
 # the file that builds its tensor maps, at capture time).
 NCU_TRAFFIC = {
-    ("prefill", "ffn_up_gemm"): {"bytes_per_launch": 37_801_926_400, "src": "62105494cf85"},
-    ("decode", "ffn_up_gemm"): {"bytes_per_launch": 7_315_725_824, "src": "62105494cf85"},
+    ("prefill", "ffn_up_gemm"): {"bytes_per_launch": 36872081152, "src": "155560179a03"},
+    ("decode", "ffn_up_gemm"): {"bytes_per_launch": 7316855552, "src": "155560179a03"},
 }
 
 
