@@ -17,6 +17,7 @@ is the maximum over ranks.
 import argparse
 import datetime
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -44,11 +45,11 @@ LAUNCHES_PER_STEP = 10  # router GEMM, top-K, histogram, scan, permute, gather, 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM traffic per launch of the dominant kernel from an ncu capture (profiles/), valid only
-# while the kernel and its launch set-up are unchanged (sha1 of the GEMM kernel source and of
-# the file that builds its tensor maps, at capture time).
+# while the kernel and its launch set-up are unchanged (sha1 of the code, comments removed, of
+# the GEMM kernel and of the file that builds its tensor maps, at capture time).
 NCU_TRAFFIC = {
-    ("prefill", "ffn_up_gemm"): {"bytes_per_launch": 36872081152, "src": "155560179a03"},
-    ("decode", "ffn_up_gemm"): {"bytes_per_launch": 7316855552, "src": "155560179a03"},
+    ("prefill", "ffn_up_gemm"): {"bytes_per_launch": 36872081152, "src": "0652bf0f6854"},
+    ("decode", "ffn_up_gemm"): {"bytes_per_launch": 7316855552, "src": "0652bf0f6854"},
 }
 
 
@@ -65,11 +66,23 @@ def peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def gemm_source_hash():
+def _code_only(text):
+    """C/C++ source without comments and blank space, so comment edits keep the hash."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.strip() for line in text.splitlines() if line.strip())
+
+
+def gemm_source_hash(read=None):
     h = hashlib.sha1()
     for name in ("gemm.cu", "device.cuh", "kernels.cuh", "moe_api.cu"):
-        with open(os.path.join(ROOT, "mixture_experts_layer_38_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        path = os.path.join("mixture_experts_layer_38_b200", "csrc", name)
+        if read is None:
+            with open(os.path.join(ROOT, path), encoding="utf-8") as f:
+                text = f.read()
+        else:
+            text = read(path)
+        h.update(_code_only(text).encode())
     return h.hexdigest()[:12]
 
 

@@ -24,6 +24,8 @@
 //               per-warp shared-memory transpose and coalesced row stores.  A warp may only
 //               read the TMEM lane quarter (warp id mod 4); with more than four epilogue warps
 //               the warps of a quarter take alternate 32-token chunks of the tile.
+//   warps 6-13  FP8-weight instantiations only: converters (E4M3 codes -> bf16 slots, see Cfg)
+//   warps 6-9   row-gather instantiation only: token-row loaders (cp.async, see Cfg)
 // Token tiles come in two kinds: full 128-row tiles (compute-bound) and each expert's partial
 // tail tile (for the many lightly loaded experts: weight streaming).  The static schedule
 // interleaves the two lists in proportion, and within a token tile the weight tiles come
@@ -64,7 +66,7 @@ constexpr int kSmemPrefix = 2 * (kMaxGroups + 4) * 4;  // full-tile and tail-til
 //
 // FP8 weights (WQ, used with BN = 128): a stage holds the two weight blocks as E4M3 codes
 // (2 x 8 KB, half the bytes, so twice the weights in flight per byte of ring) and the token
-// rows; eight converter warps (one block each per group of four) turn the codes into bf16
+// rows; eight converter warps (four per weight block) turn the codes into bf16
 // (times the block's power-of-two scale: exact) in a separate ring of two 32 KB bf16 slots,
 // which is what the MMA reads.  A stage is free again once the converters have read its
 // codes and the MMA its token rows; a slot once the MMA has read it.
