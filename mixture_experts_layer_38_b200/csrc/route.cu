@@ -24,6 +24,7 @@ namespace {
 // Selection key of expert id with score s:
 // (order-preserving bits of s) << 32 | (0xffffffff - id)  ->  larger score, then lower id.
 constexpr int kBlockThreads = 256;
+constexpr int kWarps = kBlockThreads / 32;
 constexpr int kMaxPerThread = 4;  // E <= 1024
 
 __device__ __forceinline__ uint64_t score_key(float s, int id) {
@@ -65,7 +66,7 @@ __global__ void __launch_bounds__(kBlockThreads, kPerThread <= 3 ? 4 : 3)
                             int32_t *__restrict__ topk_idx, float *__restrict__ topk_gate,
                             float *__restrict__ gap, int *status) {
   __shared__ float red[kBlockThreads / 32];
-  __shared__ uint64_t wbest[kBlockThreads / 32];
+  __shared__ uint64_t wbest[2][kWarps];
   __shared__ int sel_id[33];
   __shared__ float sel_p[33];
   __shared__ float sel_s[33];
@@ -105,15 +106,23 @@ __global__ void __launch_bounds__(kBlockThreads, kPerThread <= 3 ? 4 : 3)
     key[j] = (e < E) ? score_key(__fadd_rn(p[j], __ldg(b + e)), e) : 0ull;
   }
   const int rounds = K < E ? K + 1 : K;
+  // One barrier per round: the warp maxima alternate between two buffers, so round k + 2
+  // cannot overwrite what a slow thread still reads from round k (every thread passes round
+  // k + 1's barrier first).
   for (int k = 0; k < rounds; ++k) {
+    uint64_t *wb = wbest[k & 1];
     uint64_t best = key[0];
 #pragma unroll
     for (int j = 1; j < kPerThread; ++j) best = key[j] > best ? key[j] : best;
     best = warp_max_u64(best);
-    if ((tid & 31) == 0) wbest[tid >> 5] = best;
+    if ((tid & 31) == 0) wb[tid >> 5] = best;
     __syncthreads();
-    uint64_t win = wbest[0];
-    for (int w = 1; w < kBlockThreads / 32; ++w) win = wbest[w] > win ? wbest[w] : win;
+    uint64_t win = wb[tid & (kWarps - 1)];  // lane i takes warp i % 8's maximum
+#pragma unroll
+    for (int off = 1; off < kWarps; off <<= 1) {
+      const uint64_t o = __shfl_xor_sync(0xffffffffu, win, off);
+      win = o > win ? o : win;
+    }
     const int id = (int)(0xffffffffu - (uint32_t)(win & 0xffffffffu));
     if (win == 0ull) {  // nothing left that is selectable (non-finite scores): flag, skip
       if (tid == 0) {
@@ -133,8 +142,8 @@ __global__ void __launch_bounds__(kBlockThreads, kPerThread <= 3 ? 4 : 3)
         }
       }
     }
-    __syncthreads();
   }
+  __syncthreads();  // the selections of the last round are written
   if (tid < 32) {
     const int lane = tid;
     const int my_id = lane < K ? sel_id[lane] : 0x7fffffff;
