@@ -612,7 +612,10 @@ int moe_forward_timed(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *W
 int moe_quantize_fp8(const moe_bf16 *w, int64_t G, int64_t R, int64_t C, uint8_t *q,
                      float *scale, void *stream) {
   MOE_REQUIRE(G >= 0 && R >= 0 && C >= 0 && R % 128 == 0 && C % 128 == 0, MOE_ERR_SHAPE);
-  MOE_REQUIRE(G == 0 || R == 0 || C == 0 || G * (R / 128) * (C / 128) < (1ll << 31),
+  MOE_REQUIRE(G < (1ll << 31) && R < (1ll << 31) && C < (1ll << 31), MOE_ERR_SHAPE);
+  // one CTA per 128 x 128 block: the block count must fit a grid dimension
+  MOE_REQUIRE(G == 0 || R == 0 || C == 0 ||
+                  (R / 128) * (C / 128) <= ((1ll << 31) - 1) / G,
               MOE_ERR_SHAPE);
   if (G == 0 || R == 0 || C == 0) return MOE_OK;
   MOE_CHECK_PTR(w);

@@ -94,6 +94,8 @@ def test_fp8_shape_errors_before_device_work():
     assert lib.moe_quantize_fp8(P(0x10000), 1, 100, 128, P(0x20000), P(0x30000), None) == 2
     assert lib.moe_quantize_fp8(P(0x10000), 1, 128, 192, P(0x20000), P(0x30000), None) == 2
     assert lib.moe_quantize_fp8(None, 0, 128, 128, None, None, None) == 0  # nothing to do
+    assert lib.moe_quantize_fp8(P(0x10000), 1 << 40, 1 << 30, 128, P(0x20000), P(0x30000),
+                                None) == 2  # too many blocks (and no overflow in the check)
     # d = 192 is a valid bf16 width but not a whole number of 128-wide scale blocks
     dm = mb.dims(64, 192, 8, 4, 3, 256)
     args = [P(0x10000 * (i + 1)) for i in range(10)]  # x, W_r, b, 6 FP8 tensors, y
