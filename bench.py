@@ -282,6 +282,33 @@ def run_ours(args, rank, world, local_rank):
     ws = mb.alloc_workspace(dm, device)
     y = torch.empty((w.T, w.d), dtype=torch.bfloat16, device=device)
     b = wt["b"].clone()
+    dense = None
+    if args.scmoe > 0:
+        # ScMoE shortcut branch: a dense SwiGLU FFN on its own input, on a second stream
+        g = torch.Generator(device=device).manual_seed(args.seed + 77)
+        Id = args.scmoe
+        dense = {
+            "dm": mb.dims(w.T, w.d, 1, 0, 1, Id),
+            "x": torch.randn((w.T, w.d), generator=g, device=device).to(torch.bfloat16),
+            "W_g": (torch.randn((Id, w.d), generator=g, device=device) * 0.02).to(torch.bfloat16),
+            "W_u": (torch.randn((Id, w.d), generator=g, device=device) * 0.02).to(torch.bfloat16),
+            "W_d": (torch.randn((w.d, Id), generator=g, device=device) * 0.02).to(torch.bfloat16),
+            "h": torch.empty((w.T, Id), dtype=torch.bfloat16, device=device),
+            "y": torch.empty((w.T, w.d), dtype=torch.bfloat16, device=device),
+            "ws": torch.zeros(256, dtype=torch.uint8, device=device),
+            "stream": torch.cuda.Stream(device=device),
+        }
+
+    def dense_fork(main):
+        if dense is not None:
+            dense["stream"].wait_stream(main)
+            mb.moe_dense_ffn(dense["dm"], dense["x"], dense["W_g"], dense["W_u"], dense["W_d"],
+                             dense["h"], dense["y"], dense["ws"], stream=dense["stream"])
+
+    def dense_join(main):
+        if dense is not None:
+            main.wait_stream(dense["stream"])
+
     fw = None
     if args.fp8:
         log(f"[rank {rank}] quantising the expert weights to block-wise FP8")
@@ -309,12 +336,33 @@ def run_ours(args, rank, world, local_rank):
             e.record(stream)
 
     def step(i, ev=None):
+        dense_fork(stream)
         forward(x, y, counts[i], ev)
         mb.moe_bias_update(dm, counts[i], b, pid_state, params)
+        dense_join(stream)
 
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
+    scmoe = None
+    if dense is not None:  # each branch alone, for the overlap report (outside the timed region)
+        def alone(fn, n=5):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(n):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1) / n
+        scratch_counts = torch.zeros(w.E, dtype=torch.int32, device=device)
+        scmoe = {
+            "I_dense": args.scmoe,
+            "dense_ffn_ms_alone": round(alone(lambda: mb.moe_dense_ffn(
+                dense["dm"], dense["x"], dense["W_g"], dense["W_u"], dense["W_d"], dense["h"],
+                dense["y"], dense["ws"], stream=stream)), 4),
+            "moe_forward_ms_alone": round(alone(lambda: forward(x, y, scratch_counts)), 4),
+            "dense_flop_per_step": 6 * w.T * w.d * args.scmoe,
+        }
     if world > 1:
         torch.distributed.barrier()
     clocks = ClockSampler(device)
@@ -381,6 +429,9 @@ def run_ours(args, rank, world, local_rank):
     roof["kernel"] = kernel
     roof["peak_source"] = f"{pk_src} {peak_name}"
     layer_flops = sum(tot_flops.values())
+    if scmoe is not None:
+        scmoe["step_ms"] = round(ms / args.steps, 4)
+        layer_flops += scmoe["dense_flop_per_step"] * args.steps
     layer_tflops = layer_flops / (ms / 1e3) / 1e12
     layer_gbs = sum(tot_bytes.values()) / (ms / 1e3) / 1e9
     routing = (A_steps, U_steps, load_ratio)
@@ -390,6 +441,8 @@ def run_ours(args, rank, world, local_rank):
              "gbs": round(layer_gbs, 1),
              "frac_of_hbm_peak": round(layer_gbs / pk["hbm_gbs"], 4),
              "frac_of_nominal_hbm": round(layer_gbs / NOMINAL_HBM_GBS, 4)}
+    if scmoe is not None:
+        layer["scmoe"] = scmoe
 
     # ---------------------------------------------------------------- end to end, host buffers
     if args.no_e2e:
@@ -428,8 +481,10 @@ def run_ours(args, rank, world, local_rank):
             if i >= 2:
                 cs.wait_event(d2h_done[cur])  # y_dev[cur] of step i-2 has left the device
             c = counts[n_steps + (i % args.steps)]
+            dense_fork(cs)
             forward(x_dev[cur], y_dev[cur], c, stream=cs)
             mb.moe_bias_update(dm, c, b, pid_state, params, stream=cs)
+            dense_join(cs)
             comp_done[cur].record(cs)
             ds.wait_event(comp_done[cur])
             with torch.cuda.stream(ds):
@@ -473,7 +528,8 @@ def finish(args, w, world, rank, ms_max, routing, roof, layer, stage_ms, clk, e2
                     % ((w.pid_target,) + PID_GAINS),
             "variant": {"renormalize_gates": bool(args.renormalize_gates),
                         "balance_gamma": args.balance_gamma,
-                        "expert_weights": "fp8 e4m3, 128x128 blocks" if args.fp8 else "bf16"},
+                        "expert_weights": "fp8 e4m3, 128x128 blocks" if args.fp8 else "bf16",
+                        "scmoe_dense_ffn": args.scmoe or None},
             "mean_ffn_experts_per_token": round(float(np.mean(A_steps)) / w.T, 4),
             "distinct_ffn_experts": int(np.mean(U_steps)),
             "ffn_load_max_over_mean": round(float(np.mean(load_ratio)), 2),
@@ -483,7 +539,7 @@ def finish(args, w, world, rank, ms_max, routing, roof, layer, stage_ms, clk, e2
         "stages_ms": {k: round(v / args.steps, 4) for k, v in stage_ms.items()},
         "clocks": clk,
         "e2e": e2e,
-        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "gpu_launches": (LAUNCHES_PER_STEP + (2 if args.scmoe else 0)) * args.steps,
     }
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         n = args.cpu_sample or default_sample(w)
@@ -551,6 +607,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg (profiling)")
     ap.add_argument("--renormalize-gates", action="store_true",
                     help="variant: gates renormalised over the K selected experts")
+    ap.add_argument("--scmoe", type=int, default=0, metavar="I_DENSE",
+                    help="variant: a dense SwiGLU FFN of this intermediate width (the ScMoE "
+                         "shortcut branch) on a second stream beside each step")
     ap.add_argument("--fp8", action="store_true",
                     help="variant: block-wise FP8 (E4M3) expert weights, quantised on the GPU")
     ap.add_argument("--balance-gamma", type=float, default=0.0,

@@ -180,6 +180,20 @@ int moe_expert_ffn_gather(const moe_dims *dims, const moe_bf16 *x, const int32_t
                           const moe_bf16 *W_u, const moe_bf16 *W_d, moe_bf16 *h,
                           moe_bf16 *y_perm, void *ws, size_t ws_bytes, void *stream);
 
+/* Dense SwiGLU FFN, y = W_d (silu(W_g x) * (W_u x)) for every token: the shortcut branch of
+ * ScMoE ("衝上熱搜！美團大模型，靠「快」火了", §快捷連接 MoE: the previous block's dense FFN runs
+ * in parallel with the current MoE layer, which on one GPU means on a second stream beside
+ * moe_forward; the MoE layer and this call share no buffers, so they may overlap).  Uses the
+ * experts' grouped GEMMs with one group of T rows and gate 1.  Only dims->T, d and I are read
+ * (I = the dense intermediate width; d and I positive multiples of 64).
+ *   x [T, d] bf16; W_g, W_u [I, d] bf16; W_d [d, I] bf16
+ *   h [T, I] bf16 (out, scratch)    y [T, d] bf16 (out)
+ *   ws: a workspace of at least 256 bytes, first 256 zero (its status word is used); do not
+ *   share it with a concurrent moe_forward. */
+int moe_dense_ffn(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *W_g,
+                  const moe_bf16 *W_u, const moe_bf16 *W_d, moe_bf16 *h, moe_bf16 *y, void *ws,
+                  size_t ws_bytes, void *stream);
+
 /* Combine / un-permute: y_t = sum over FFN slots k (ascending expert id) of y_perm[slot_pos]
  * + (sum of the zero-expert gates of t) * x_t, accumulated in fp32 in that fixed order and
  * rounded once to bf16.  Zero experts are identities ("衝上熱搜！美團大模型，靠「快」火了",

@@ -19,7 +19,7 @@ EXPORTS = (
     "moe_strerror", "moe_workspace_size", "moe_scratch_size", "moe_route", "moe_dispatch",
     "moe_expert_ffn", "moe_combine", "moe_bias_update", "moe_forward", "moe_forward_timed",
     "moe_last_device_error", "moe_dispatch_noalloc", "moe_expert_ffn_gather",
-    "moe_quantize_fp8", "moe_expert_ffn_fp8", "moe_forward_fp8",
+    "moe_quantize_fp8", "moe_expert_ffn_fp8", "moe_forward_fp8", "moe_dense_ffn",
 )
 NUM_STAGE_EVENTS = 7
 STAGE_NAMES = ("router_gemm", "route_topk", "dispatch", "ffn_up_gemm", "ffn_down_gemm",
@@ -84,13 +84,15 @@ def lib():
         L.moe_expert_ffn_gather.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]
         _I64 = ctypes.c_int64
         L.moe_quantize_fp8.argtypes = [_P, _I64, _I64, _I64, _P, _P, _P]
+        L.moe_dense_ffn.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, _S, _P]
         L.moe_expert_ffn_fp8.argtypes = [_DP] + [_P] * 11 + [_P, _S, _P]
         L.moe_forward_fp8.argtypes = [_DP] + [_P] * 11 + [_P, _S,
                                                           ctypes.POINTER(ctypes.c_void_p), _P]
         for f in ("moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine",
                   "moe_bias_update", "moe_forward", "moe_forward_timed",
                   "moe_last_device_error", "moe_dispatch_noalloc", "moe_expert_ffn_gather",
-                  "moe_quantize_fp8", "moe_expert_ffn_fp8", "moe_forward_fp8"):
+                  "moe_quantize_fp8", "moe_expert_ffn_fp8", "moe_forward_fp8",
+                  "moe_dense_ffn"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -349,3 +351,14 @@ def moe_forward_fp8(dm, x, W_r, b, fw, y, counts, ws, stream=None, events=None):
         _ptr(counts, torch.int32, (dm.N + dm.Z,), "counts", nullable=True), w, n, ev,
         _stream(stream))
     _check("moe_forward_fp8", rc)
+
+
+def moe_dense_ffn(dm, x, W_g, W_u, W_d, h, y, ws, stream=None):
+    """Dense SwiGLU FFN of all T tokens (dm.T, dm.d, dm.I; W_g, W_u [I, d], W_d [d, I])."""
+    w, n = _ws(ws)
+    rc = lib().moe_dense_ffn(
+        ctypes.byref(dm), _ptr(x, torch.bfloat16, (dm.T, dm.d), "x"),
+        _ptr(W_g, torch.bfloat16, (dm.I, dm.d), "W_g"), _ptr(W_u, torch.bfloat16, (dm.I, dm.d), "W_u"),
+        _ptr(W_d, torch.bfloat16, (dm.d, dm.I), "W_d"), _ptr(h, torch.bfloat16, (dm.T, dm.I), "h"),
+        _ptr(y, torch.bfloat16, (dm.T, dm.d), "y"), w, n, _stream(stream))
+    _check("moe_dense_ffn", rc)

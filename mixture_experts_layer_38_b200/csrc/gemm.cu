@@ -300,7 +300,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs &a, const Tile &t,
     float gate = 0.f;
     if (EPI == kEpiGated) {
       const int tok = tok0 + lane;
-      gate = tok < t.n_valid ? __ldg(a.row_scale + t.row0 + tok) : 0.f;
+      gate = tok >= t.n_valid ? 0.f : (a.row_scale ? __ldg(a.row_scale + t.row0 + tok) : 1.f);
     }
 #pragma unroll 1
     for (int sub = 0; sub < 2; ++sub) {

@@ -32,7 +32,7 @@ struct GemmArgs {
   void *out;
   int out_ld;                    // elements per output row
   long long split_stride;        // elements between split-K partial outputs
-  const float *row_scale;        // kEpiGated: per-row gate
+  const float *row_scale;        // kEpiGated: per-row gate (NULL: 1)
   int *status;                   // device status word
   // Row gather (up-projection only): when row_index is set, activation row r is row
   // row_index[r] of the row-major bf16 matrix gather_src (K columns), copied by loader warps;

@@ -487,6 +487,69 @@ int moe_expert_ffn_gather(const moe_dims *dims, const moe_bf16 *x, const int32_t
                        static_cast<cudaStream_t>(stream), nullptr, x, perm_tok);
 }
 
+int moe_dense_ffn(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *W_g,
+                  const moe_bf16 *W_u, const moe_bf16 *W_d, moe_bf16 *h, moe_bf16 *y, void *ws,
+                  size_t ws_bytes, void *stream) {
+  MOE_REQUIRE(dims != nullptr, MOE_ERR_ARG);
+  const moe_dims &d = *dims;
+  MOE_REQUIRE(d.T >= 0 && d.d > 0 && d.d % 64 == 0 && d.I > 0 && d.I % 64 == 0 &&
+                  (long long)d.T * d.I < (1ll << 31) && (long long)d.T * d.d < (1ll << 31),
+              MOE_ERR_SHAPE);
+  MOE_CHECK_TOKEN_PTR(x, d.T);
+  MOE_CHECK_PTR(W_g);
+  MOE_CHECK_PTR(W_u);
+  MOE_CHECK_PTR(W_d);
+  MOE_CHECK_TOKEN_PTR(h, d.T);
+  MOE_CHECK_TOKEN_PTR(y, d.T);
+  int rc = check_ws(ws, ws_bytes, kAlign);
+  if (rc != MOE_OK) return rc;
+  const DeviceInfo *di = nullptr;
+  rc = device_info(&di);
+  if (rc != MOE_OK) return rc;
+  if (d.T == 0) return MOE_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int *status = at<int>(ws, 0);
+  // One group of all T rows through the same grouped GEMMs as the experts (gate 1).
+  const int tile_tokens = gemm_tile_tokens(d.T, 1, d.d);
+  const bool p256 = tile_tokens != 256;
+  GemmArgs up{};
+  if (!make_map(&up.map_a0, W_g, (uint64_t)d.I, (uint64_t)d.d, 128, p256) ||
+      !make_map(&up.map_a1, W_u, (uint64_t)d.I, (uint64_t)d.d, 128, p256) ||
+      !make_map(&up.map_a01, W_g, (uint64_t)d.I, (uint64_t)d.d, 256, p256) ||
+      !make_act_maps(up, x, (uint64_t)d.T, (uint64_t)d.d, p256)) {
+    return MOE_ERR_CUDA;
+  }
+  up.group_offsets = nullptr;
+  up.num_groups = 1;
+  up.rows = d.T;
+  up.M = d.I;
+  up.K = d.d;
+  up.k_splits = 1;
+  up.out = h;
+  up.out_ld = d.I;
+  up.status = status;
+  if (launch_grouped_gemm(kEpiSwiGLU, up, di->sms, tile_tokens, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  GemmArgs down{};
+  if (!make_map(&down.map_a0, W_d, (uint64_t)d.d, (uint64_t)d.I, 128, p256) ||
+      !make_map(&down.map_a1, W_d, (uint64_t)d.d, (uint64_t)d.I, 128, p256) ||
+      !make_map(&down.map_a01, W_d, (uint64_t)d.d, (uint64_t)d.I, 256, p256) ||
+      !make_act_maps(down, h, (uint64_t)d.T, (uint64_t)d.I, p256)) {
+    return MOE_ERR_CUDA;
+  }
+  down.group_offsets = nullptr;
+  down.num_groups = 1;
+  down.rows = d.T;
+  down.M = d.d;
+  down.K = d.I;
+  down.k_splits = 1;
+  down.out = y;
+  down.out_ld = d.d;
+  down.row_scale = nullptr;  // gate 1
+  down.status = status;
+  return to_status(launch_grouped_gemm(kEpiGated, down, di->sms, tile_tokens, s));
+}
+
 int moe_combine(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *y_perm,
                 const int32_t *topk_idx, const float *topk_gate, const int32_t *slot_pos,
                 moe_bf16 *y, void *stream) {

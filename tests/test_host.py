@@ -107,6 +107,19 @@ def test_fp8_shape_errors_before_device_work():
                                mb.workspace_size(dm2), None, None) == 1
 
 
+def test_dense_ffn_argument_errors():
+    lib = mb.lib()
+    for bad in [(64, 100, 1, 0, 1, 256), (64, 128, 1, 0, 1, 96), (-1, 128, 1, 0, 1, 256)]:
+        dm = mb.dims(*bad)
+        assert lib.moe_dense_ffn(ctypes.byref(dm), *[P(0x10000)] * 6, P(0x100000), 256,
+                                 None) == 2
+    dm = mb.dims(64, 128, 1, 0, 1, 256)
+    assert lib.moe_dense_ffn(ctypes.byref(dm), P(0x10000), P(0), P(0x10000), P(0x10000),
+                             P(0x10000), P(0x10000), P(0x100000), 256, None) == 1
+    assert lib.moe_dense_ffn(ctypes.byref(dm), *[P(0x10000)] * 6, P(0x100000), 128,
+                             None) == 4  # workspace smaller than its 256-byte status region
+
+
 def test_variant_switches_are_validated():
     lib = mb.lib()
     dm = mb.dims(64, 128, 8, 4, 3, 256, flags=mb.RENORMALIZE_GATES)
