@@ -15,8 +15,13 @@
 // the gate and the up value of one feature and SwiGLU needs no data exchange.  For the down
 // projection and the router they are 256 consecutive output rows.
 //
+// 256-token tiles of the FFN GEMMs run on CTA pairs (Cfg, PR): a cluster of two CTAs on two
+// SMs issues pair MMAs of M = 256 weight rows, each CTA holding half the weight rows and half
+// the token rows of a stage, so a third less shared memory feeds the same work per SM.
+//
 // Warp roles (64 + 32 x kGemmEpiWarps = 192 threads, one CTA per SM, persistent over a static
-// tile schedule):
+// tile schedule; with CTA pairs only the even CTA's warp 1 issues MMAs, whose commits signal
+// both CTAs, and both CTAs' epilogues release the accumulator on the even CTA's barrier):
 //   warp 0      TMA producer: A0/A1 weight tiles (128 x 64) and the token tile (n x 64, issued
 //               as 256/128/64/32/16-row boxes) into a 192 KB ring of 48 KB or 64 KB stages
 //   warp 1      TMEM allocator (512 columns: 2 buffers x 2 x 128, or 1 x 2 x 256) and MMA issuer
@@ -78,10 +83,17 @@ constexpr int kConvWarps = 8;
 constexpr int kLoadWarps = 4;
 constexpr int kLoadThreads = 32 * kLoadWarps;
 
-template <int BN, bool WQ = false, bool GA = false>
+// CTA pairs (PR, used with BN = 256): a cluster of two CTAs on two SMs computes a tile of
+// 2 x 256 weight rows x up to 256 tokens with pair MMAs (M = 256).  CTA r holds weight rows
+// [128 r, 128 r + 128) of each 256-row sub-tile and token rows [r nb/2, (r+1) nb/2) of the tile
+// in its own 48 KB stages (4 in the ring); the even CTA issues the MMAs, which read both CTAs'
+// operands and leave each CTA's 128 rows x nb columns in its own TMEM.  Per SM and k-step,
+// 48 KB of shared memory feed the work that takes 64 KB in a single-CTA 256-token tile.
+template <int BN, bool WQ = false, bool GA = false, bool PR = false>
 struct Cfg {
+  static_assert(!PR || (BN == 256 && !WQ && !GA), "CTA pairs: 256-token tiled loads only");
   static constexpr int kAccBufs = BN <= 128 ? 2 : 1;
-  static constexpr int kStage = (WQ ? 2 * kQTile : 2 * kTileA) + BN * kBK * 2;
+  static constexpr int kStage = (WQ ? 2 * kQTile : 2 * kTileA) + (PR ? BN / 2 : BN) * kBK * 2;
   static constexpr int kCSlots = WQ ? 2 : 0;              // bf16 weight slots
   static constexpr int kCRing = kCSlots * 2 * kTileA;
   static constexpr int kStages = (192 * 1024 - kCRing) / kStage;
@@ -137,8 +149,9 @@ __device__ __forceinline__ int find_group(const int *pre, int G, int v) {
   return lo;
 }
 
-template <int EPI, int BN>
-__device__ __forceinline__ Tile decode_tile(const GemmArgs &a, const Schedule &s, int tile) {
+template <int EPI, int BN, bool PR = false>
+__device__ __forceinline__ Tile decode_tile(const GemmArgs &a, const Schedule &s, int tile,
+                                            uint32_t rank = 0) {
   Tile t;
   const int mt = tile % s.m_tiles;
   const int rest = tile / s.m_tiles;
@@ -161,17 +174,18 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs &a, const Schedule &s
     t.n_valid = BN;
     t.once = false;
   }
-  t.nb = (t.n_valid + 15) & ~15;
+  // A pair MMA splits N in two halves of a multiple of 16 rows each.
+  t.nb = PR ? (t.n_valid + 31) & ~31 : (t.n_valid + 15) & ~15;
   if (EPI == kEpiSwiGLU) {
-    t.m0 = mt * kBM;
+    t.m0 = PR ? mt * 2 * kBM + (int)rank * kBM : mt * kBM;
     t.a0_row = g * a.M + t.m0;
     t.a1_row = t.a0_row;
     t.has_a1 = true;
   } else {
-    t.m0 = mt * 2 * kBM;
+    t.m0 = PR ? mt * 4 * kBM + (int)rank * 2 * kBM : mt * 2 * kBM;
     t.a0_row = g * a.M + t.m0;
     t.a1_row = t.a0_row + kBM;
-    t.has_a1 = (t.m0 + kBM) < a.M;
+    t.has_a1 = PR || (t.m0 + kBM) < a.M;  // a pair always fills both (M divides evenly)
   }
   const int kblocks = a.K / kBK;
   t.kb0 = (int)(((long long)kblocks * t.split) / s.splits);
@@ -245,9 +259,10 @@ __device__ bool build_schedule(const GemmArgs &a, int *hpre, int *lpre, int *scr
   return !any_bad;
 }
 
-template <int EPI>
+template <int EPI, bool PR = false>
 __device__ __forceinline__ int m_tiles_of(int M) {
-  return EPI == kEpiSwiGLU ? (M + kBM - 1) / kBM : (M + 2 * kBM - 1) / (2 * kBM);
+  const int rows = (EPI == kEpiSwiGLU ? kBM : 2 * kBM) * (PR ? 2 : 1);
+  return (M + rows - 1) / rows;
 }
 
 // Bounded wait by lane 0 of a warp, result broadcast so the warp stays converged.
@@ -384,10 +399,10 @@ __device__ __forceinline__ void convert_fp8_block(const uint8_t *q, uint8_t *dst
   }
 }
 
-template <int EPI, int BN, bool WQ, bool GATHER>
-__global__ void __launch_bounds__(Cfg<BN, WQ, GATHER>::kThreads, 1)
+template <int EPI, int BN, bool WQ, bool GATHER, bool PR = false>
+__global__ void __launch_bounds__(Cfg<BN, WQ, GATHER, PR>::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ GemmArgs args) {
-  using C = Cfg<BN, WQ, GATHER>;
+  using C = Cfg<BN, WQ, GATHER, PR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -410,6 +425,10 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER>::kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // Tiles are dealt to CTAs, or with CTA pairs to pairs (both CTAs walk the same tiles).
+  const uint32_t rank = PR ? cluster_ctarank() : 0u;
+  const int unit = PR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int units = PR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -418,7 +437,7 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER>::kThreads, 1)
     }
     for (int b = 0; b < C::kAccBufs; ++b) {
       mbar_init(&tfull_bar[b], 1);
-      mbar_init(&tempty_bar[b], kEpiWarps);
+      mbar_init(&tempty_bar[b], (PR ? 2 : 1) * kEpiWarps);  // PR: both CTAs' epilogues
     }
     mbar_init(drain_bar, 1);
     for (int c = 0; c < C::kCSlots; ++c) {
@@ -437,16 +456,22 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER>::kThreads, 1)
     for (int i = 0; i < 4; ++i) tma_prefetch_desc(&args.map_b[i]);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
+    if (PR) {
+      tmem_alloc_pair(tmem_slot, kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, kTmemCols);
+      tmem_relinquish();
+    }
   }
   Schedule sched;
   build_schedule<BN>(args, hpre, lpre, reinterpret_cast<int *>(staging), sched);
-  sched.m_tiles = m_tiles_of<EPI>(args.M);
+  sched.m_tiles = m_tiles_of<EPI, PR>(args.M);
   sched.splits = EPI == kEpiF32 ? args.k_splits : 1;
   sched.total = sched.total * sched.m_tiles * sched.splits;
   tc_fence_before();
-  __syncthreads();
+  if (PR) cluster_sync();  // both CTAs' barriers initialised before any remote arrival
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -464,10 +489,12 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER>::kThreads, 1)
       uint32_t phase = 0;
       long long issued = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < sched.total; tile += gridDim.x) {
-        const Tile t = decode_tile<EPI, BN>(args, sched, tile);
-        const uint32_t bytes = (WQ ? kQTile : kTileA) * (t.has_a1 ? 2 : 1) +
-                               (GATHER ? 0 : t.nb * kBK * 2);
+      for (int tile = unit; ok && tile < sched.total; tile += units) {
+        const Tile t = decode_tile<EPI, BN, PR>(args, sched, tile, rank);
+        // PR: the even CTA's stage barrier counts both CTAs' bytes (equal halves).
+        const uint32_t bytes = PR ? 2u * (2 * kTileA + (t.nb / 2) * kBK * 2)
+                                  : (WQ ? kQTile : kTileA) * (t.has_a1 ? 2 : 1) +
+                                        (GATHER ? 0 : t.nb * kBK * 2);
         const uint64_t pol_w = t.once ? pol_w_once : pol_w_reused;
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag)) {
@@ -479,6 +506,29 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER>::kThreads, 1)
           uint8_t *sa1 = sa0 + kTileA;
           uint8_t *sb = sa0 + (WQ ? 2 * kQTile : 2 * kTileA);
           const int kc = kb * kBK;
+          if (PR) {
+            const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
+            if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], bytes);
+            if (EPI != kEpiSwiGLU) {
+              tma_load_2d_pair(sa0, &args.map_a01, fb, kc, t.a0_row, pol_w);
+            } else {
+              tma_load_2d_pair(sa0, &args.map_a0, fb, kc, t.a0_row, pol_w);
+              tma_load_2d_pair(sa1, &args.map_a1, fb, kc, t.a1_row, pol_w);
+            }
+            const int half = t.nb >> 1, brow = t.row0 + (int)rank * half;
+            int r = 0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int box = 128 >> i;
+              if (half - r >= box) {
+                tma_load_2d_pair(sb + r * (kBK * 2), &args.map_b[i], fb, kc, brow + r, pol_x);
+                r += box;
+              }
+            }
+            ++issued;
+            if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+            continue;
+          }
           mbar_arrive_expect_tx(&full_bar[stage], bytes);
           if (WQ) {  // E4M3 codes of both weight blocks at the start of the stage
             tma_load_2d(sa0, &args.map_a0, &full_bar[stage], kc, t.a0_row, pol_w);
@@ -515,8 +565,9 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER>::kThreads, 1)
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
         }
       }
-      if (!ok) {
-        // Drain the copies that may still be landing in the ring (bounded).
+      if (!ok && !(PR && rank != 0)) {
+        // Drain the copies that may still be landing in the ring (bounded; with CTA pairs the
+        // even CTA's barriers count both CTAs' copies).
         for (long long i = 1; i <= issued && i <= C::kStages; ++i) {
           const long long idx = issued - i;
           const int s = (int)(idx % C::kStages);
@@ -528,7 +579,7 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER>::kThreads, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       int stage = 0;
       uint32_t phase = 0;
       int cslot = 0;            // WQ: bf16 slot of the current k-step
@@ -536,8 +587,8 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER>::kThreads, 1)
       int it = 0;
       bool ok = true;
       bool any = false;
-      for (int tile = blockIdx.x; ok && tile < sched.total; tile += gridDim.x, ++it) {
-        const Tile t = decode_tile<EPI, BN>(args, sched, tile);
+      for (int tile = unit; ok && tile < sched.total; tile += units, ++it) {
+        const Tile t = decode_tile<EPI, BN, PR>(args, sched, tile, rank);
         const int buf = it % C::kAccBufs;
         const uint32_t use = (uint32_t)(it / C::kAccBufs);
         if (!mbar_wait(&tempty_bar[buf], (use & 1) ^ 1, abort_flag)) {
@@ -548,7 +599,7 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER>::kThreads, 1)
         tc_fence_after();
         const uint32_t d0 = tmem_base + buf * (2 * BN);
         const uint32_t d1 = d0 + BN;
-        const uint32_t idesc = idesc_bf16_f32(kBM, t.nb);
+        const uint32_t idesc = idesc_bf16_f32(PR ? 2 * kBM : kBM, t.nb);
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
           if (!mbar_wait(&full_bar[stage], phase, abort_flag) ||
               (WQ && !mbar_wait(&cfull_bar[cslot], cphase, abort_flag))) {
@@ -567,12 +618,18 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER>::kThreads, 1)
           for (int k = 0; k < kBK / 16; ++k) {
             const uint64_t bdesc = sw128_kmajor_desc(bbase + k * 32);
             const uint32_t acc = (kb > t.kb0 || k > 0) ? 1u : 0u;
-            umma_bf16(d0, sw128_kmajor_desc(abase + k * 32), bdesc, idesc, acc);
-            if (t.has_a1)
-              umma_bf16(d1, sw128_kmajor_desc(abase + kTileA + k * 32), bdesc, idesc, acc);
+            if (PR) {
+              umma_bf16_pair(d0, sw128_kmajor_desc(abase + k * 32), bdesc, idesc, acc);
+              umma_bf16_pair(d1, sw128_kmajor_desc(abase + kTileA + k * 32), bdesc, idesc, acc);
+            } else {
+              umma_bf16(d0, sw128_kmajor_desc(abase + k * 32), bdesc, idesc, acc);
+              if (t.has_a1)
+                umma_bf16(d1, sw128_kmajor_desc(abase + kTileA + k * 32), bdesc, idesc, acc);
+            }
           }
           any = true;
-          umma_commit(&empty_bar[stage]);
+          if (PR) umma_commit_pair(&empty_bar[stage], 0x3);  // frees the stage in both CTAs
+          else umma_commit(&empty_bar[stage]);
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
           if (WQ) {
             umma_commit(&cempty_bar[cslot]);
@@ -580,10 +637,12 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER>::kThreads, 1)
           }
         }
         if (!ok) break;
-        umma_commit(&tfull_bar[buf]);
+        if (PR) umma_commit_pair(&tfull_bar[buf], 0x3);
+        else umma_commit(&tfull_bar[buf]);
       }
       if (!ok && any) {
-        umma_commit(drain_bar);
+        if (PR) umma_commit_pair(drain_bar, 0x1);
+        else umma_commit(drain_bar);
         const long long t0 = clock64();
         while (!mbar_try_wait(drain_bar, 0) && clock64() - t0 < kDrainLimitCycles) {}
       }
@@ -599,7 +658,7 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER>::kThreads, 1)
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < sched.total; tile += gridDim.x) {
+    for (int tile = unit; ok && tile < sched.total; tile += units) {
       const Tile t = decode_tile<EPI, BN>(args, sched, tile);
       const int nrow = t.nb >> 4;  // rows of this thread: r0 + 16 * i, i < nrow (<= 16)
       int rix[16];
@@ -637,7 +696,7 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER>::kThreads, 1)
     int stage = 0, cslot = 0;
     uint32_t phase = 0, cphase = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < sched.total; tile += gridDim.x) {
+    for (int tile = unit; ok && tile < sched.total; tile += units) {
       const Tile t = decode_tile<EPI, BN>(args, sched, tile);
       const int row = half ? t.a1_row : t.a0_row;
       const float *scales = (half ? args.scale_a1 : args.scale_a0) + (row / 128) * args.scale_ld;
@@ -670,8 +729,8 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER>::kThreads, 1)
     const int group = (warp - 2) >> 2;   // the warps of a quarter take alternate 32-token chunks
     float *stage = staging + (warp - 2) * kStagingFloats;
     int it = 0;
-    for (int tile = blockIdx.x; tile < sched.total; tile += gridDim.x, ++it) {
-      const Tile t = decode_tile<EPI, BN>(args, sched, tile);
+    for (int tile = unit; tile < sched.total; tile += units, ++it) {
+      const Tile t = decode_tile<EPI, BN, PR>(args, sched, tile, rank);
       const int buf = it % C::kAccBufs;
       const uint32_t use = (uint32_t)(it / C::kAccBufs);
       if (!warp_wait(&tfull_bar[buf], use & 1, abort_flag)) {
@@ -685,23 +744,67 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER>::kThreads, 1)
         epilogue_chunk<EPI, BN>(args, t, tcol + c * 32, c, q, lane, stage);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty_bar[buf]);
+      if (lane == 0) {
+        if (PR) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty_bar[buf]), 0));
+        else mbar_arrive(&tempty_bar[buf]);
+      }
     }
   }
 
   tc_fence_before();
-  __syncthreads();
+  if (PR) {
+    __syncwarp();    // lanes 1-31 of warps 0 and 1 skipped the role loops: reconverge
+    cluster_sync();  // no CTA leaves while its peer may still touch its barriers or memory
+  } else {
+    __syncthreads();
+  }
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    if (PR) tmem_dealloc_pair(tmem_base, kTmemCols);
+    else tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 
-template <int EPI, int BN, bool WQ = false, bool GATHER = false>
+template <int EPI, int BN, bool WQ = false, bool GATHER = false, bool PR = false>
 cudaError_t set_smem_limit() {
-  return cudaFuncSetAttribute(grouped_gemm_kernel<EPI, BN, WQ, GATHER>,
+  return cudaFuncSetAttribute(grouped_gemm_kernel<EPI, BN, WQ, GATHER, PR>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              Cfg<BN, WQ, GATHER>::kSmemBytes);
+                              Cfg<BN, WQ, GATHER, PR>::kSmemBytes);
+}
+
+using PairCfg = Cfg<256, false, false, true>;
+constexpr int kMaxDevices = 64;
+int g_max_pairs[kMaxDevices] = {0};
+
+cudaLaunchConfig_t pair_config(int pairs, cudaStream_t stream, cudaLaunchAttribute *attr) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(PairCfg::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = PairCfg::kSmemBytes;
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
+// Shared-memory limit of a pair instantiation, and the pairs that can be resident at once.
+template <int EPI>
+cudaError_t prepare_pair(int device) {
+  cudaError_t e = set_smem_limit<EPI, 256, false, false, true>();
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[1];
+  const cudaLaunchConfig_t cfg = pair_config(1, nullptr, attr);
+  int clusters = 0;
+  e = cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_kernel<EPI, 256, false, false, true>,
+                                     &cfg);
+  if (e != cudaSuccess) return e;
+  if (clusters <= 0) return cudaErrorInvalidConfiguration;
+  if (g_max_pairs[device] == 0 || clusters < g_max_pairs[device]) g_max_pairs[device] = clusters;
+  return cudaSuccess;
 }
 
 template <int BN>
@@ -729,8 +832,10 @@ cudaError_t launch_bn(int epi, const GemmArgs &args, int grid, cudaStream_t stre
 }  // namespace
 
 cudaError_t gemm_prepare(int device) {
-  (void)device;
+  if (device < 0 || device >= kMaxDevices) return cudaErrorInvalidDevice;
   cudaError_t e;
+  if ((e = prepare_pair<kEpiSwiGLU>(device)) != cudaSuccess) return e;
+  if ((e = prepare_pair<kEpiGated>(device)) != cudaSuccess) return e;
   if ((e = set_smem_limit<kEpiSwiGLU, 128>()) != cudaSuccess) return e;
   if ((e = set_smem_limit<kEpiGated, 128>()) != cudaSuccess) return e;
   if ((e = set_smem_limit<kEpiF32, 128>()) != cudaSuccess) return e;
@@ -748,6 +853,27 @@ int gemm_tile_tokens(long long rows, int groups, int K) {
   // bound since zero-expert slots are counted too) and a long reduction, over which the
   // single accumulator buffer's epilogue stall is amortised.  Otherwise 128.
   return (rows >= 128ll * groups && K >= 4096) ? 256 : 128;
+}
+
+int gemm_max_pairs(int device) {
+  return (device >= 0 && device < kMaxDevices) ? g_max_pairs[device] : 0;
+}
+
+cudaError_t launch_grouped_gemm_pair(int epi, const GemmArgs &args, int pairs,
+                                     cudaStream_t stream) {
+  if (pairs <= 0) return cudaErrorInvalidConfiguration;
+  cudaLaunchAttribute attr[1];
+  const cudaLaunchConfig_t cfg = pair_config(pairs, stream, attr);
+  switch (epi) {
+    case kEpiSwiGLU:
+      return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kEpiSwiGLU, 256, false, false, true>,
+                                args);
+    case kEpiGated:
+      return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kEpiGated, 256, false, false, true>,
+                                args);
+    default:
+      return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t launch_grouped_gemm(int epi, const GemmArgs &args, int grid, int tile_tokens,

@@ -59,6 +59,12 @@ cudaError_t gemm_prepare(int device);  // sets the kernels' shared-memory limit 
 int gemm_tile_tokens(long long rows, int groups, int K);
 cudaError_t launch_grouped_gemm(int epi, const GemmArgs &args, int grid, int tile_tokens,
                                 cudaStream_t stream);
+// SwiGLU or gated grouped GEMM with 256-token tiles on CTA pairs (clusters of two SMs, pair
+// MMAs of 256 weight rows).  Needs M a multiple of 256 (SwiGLU) or 512 (gated); `pairs` = the
+// persistent pairs to launch (gemm_max_pairs caps it).
+cudaError_t launch_grouped_gemm_pair(int epi, const GemmArgs &args, int pairs,
+                                     cudaStream_t stream);
+int gemm_max_pairs(int device);  // co-resident pairs on the device (gemm_prepare queries it)
 // SwiGLU or gated grouped GEMM with E4M3 block-quantised weights, 128-token tiles.
 cudaError_t launch_grouped_gemm_fp8(int epi, const GemmArgs &args, int grid,
                                     cudaStream_t stream);

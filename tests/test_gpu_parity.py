@@ -109,6 +109,35 @@ def test_expert_ffn_matches_oracle(name):
     assert st.device_status() == 0
 
 
+@pytest.mark.parametrize("I", [512, 384])
+def test_expert_ffn_wide_tiles_matches_oracle(I):
+    # d = 4096 with >= 128 rows per expert selects 256-token tiles: I = 512 runs them on CTA
+    # pairs (I a multiple of 256, d of 512), I = 384 on single CTAs.  Ragged groups built
+    # directly: full 256-row tiles with and without tails, tail-only experts (100 / 30 / 17 /
+    # 1 rows), an empty expert; 1224 rows = 306 tokens x K = 4.
+    counts = np.array([520, 300, 256, 100, 17, 1, 0, 30])
+    R = int(counts.sum())
+    w = Workload("wide", T=R // 4, d=4096, N=8, Z=4, K=4, I=I)
+    wt = make_weights(w, seed=5)
+    xr = make_tokens(w, seed=5, T=R)
+    gates = np.random.default_rng(5).uniform(0.05, 1.0, R).astype(np.float32)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    xb = oracle.bf16_bits(xr)
+    want = np.zeros((R, w.d))
+    for e in range(w.N):
+        lo, hi = offsets[e], offsets[e + 1]
+        if hi > lo:
+            want[lo:hi] = gates[lo:hi, None].astype(np.float64) * oracle.swiglu_expert(
+                xb[lo:hi], wt["W_g"][e], wt["W_u"][e], wt["W_d"][e])
+    st = Stages(w, xr[: w.T], wt)
+    st.x_perm.copy_(xr)
+    st.offsets.copy_(torch.from_numpy(offsets))
+    st.perm_gate.copy_(torch.from_numpy(gates))
+    st.expert_ffn()
+    assert_y_close(oracle.bf16_to_f64(to_np(st.y_perm)), want, f"wide I={I} y_perm")
+    assert st.device_status() == 0
+
+
 @pytest.mark.parametrize("name,T", [("tiny", None), ("mid", 256), ("mid", 333)])
 def test_expert_ffn_gather_matches_oracle_and_unfused(name, T):
     # The up-projection gathering token rows from x by perm_tok (no x_perm): against the
