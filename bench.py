@@ -7,7 +7,8 @@ inputs resident in HBM.  Default workload: prefill (T=16384 tokens, d=6144, 512 
 of width 2048 plus 256 zero experts, K=12).  Weights (38.7 GB) and x (201 MB) are far larger
 than the 126 MB L2, so no L2 flush is needed between steps.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill|decode|skewed|mid|tiny]
+  python bench.py [--gpus N] [--steps K] [--warmup W]
+      [--workload prefill|decode|skewed|mid|tiny|prefill_small]
   python bench.py --impl reference ...     # the CPU oracle on a bounded sample, host cores
 
 With N > 1 (torchrun, one process per GPU) every rank runs an independent replica on its own

@@ -74,6 +74,10 @@ WORKLOADS = {
     "prefill": Workload("prefill", T=16384, d=6144, N=512, Z=256, K=12, I=2048),
     "skewed": Workload("skewed", T=8192, d=6144, N=512, Z=256, K=12, I=2048, zipf_s=1.1,
                        pid_steps=50, pid_target=8.0),
+    # The prefill layer's widths with a sixteenth of its experts and tokens (2.4 GB of weights,
+    # still far above the L2): the small case for multi-pass profiler captures of the
+    # 256-token-tile GEMMs.
+    "prefill_small": Workload("prefill_small", T=1536, d=6144, N=32, Z=16, K=12, I=2048),
 }
 
 _GEN_ON_DEVICE_ABOVE = 2 * 10**9
