@@ -49,8 +49,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # while the kernel and its launch set-up are unchanged (sha1 of the code, comments removed, of
 # the GEMM kernel and of the file that builds its tensor maps, at capture time).
 NCU_TRAFFIC = {
-    ("prefill", "ffn_up_gemm"): {"bytes_per_launch": 37913846784, "src": "31a8e1a4739b"},
-    ("decode", "ffn_up_gemm"): {"bytes_per_launch": 7316039680, "src": "31a8e1a4739b"},
+    ("prefill", "ffn_up_gemm"): {"bytes_per_launch": 36312271360, "src": "a1a46c489207"},
+    ("decode", "ffn_up_gemm"): {"bytes_per_launch": 7316081920, "src": "a1a46c489207"},
 }
 
 

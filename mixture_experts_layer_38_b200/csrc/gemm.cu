@@ -277,7 +277,11 @@ __device__ __forceinline__ void signal_abort(const GemmArgs &a, volatile int *ab
   *abort = 1;
 }
 
-__device__ __forceinline__ float silu(float z) { return z / (1.0f + __expf(-z)); }
+// silu(z) = z / (1 + e^-z) with the fast division: a few ulp in fp32, far below the bf16 rounding
+// of h that follows; for z below about -87 it returns 0 (the true value is under 1e-36).  The
+// epilogue runs between tiles on the MMA thread's critical path, and with the IEEE division's
+// longer sequence the up-projection took ~7% longer.
+__device__ __forceinline__ float silu(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
 // ------------------------------------------------------------------ epilogue, one 32-token chunk
 // Thread `lane` of epilogue warp with TMEM lane quarter q owns output feature (q*32 + lane) of
