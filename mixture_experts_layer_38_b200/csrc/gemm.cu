@@ -31,7 +31,7 @@
 //               the warps of a quarter take alternate 32-token chunks of the tile.
 //   warps 6-13  FP8-weight instantiations only: converters (E4M3 codes -> bf16 slots, see Cfg)
 //   warps 6-9   row-gather instantiation only: token-row loaders (cp.async, see Cfg)
-// Token tiles come in two kinds: full 128-row tiles (compute-bound) and each expert's partial
+// Token tiles come in two kinds: full tiles of BN rows (compute-bound) and each expert's partial
 // tail tile (for the many lightly loaded experts: weight streaming).  The static schedule
 // interleaves the two lists in proportion, and within a token tile the weight tiles come
 // fastest, so the CTAs in flight share token tiles and walk one expert's weights together (L2
