@@ -40,8 +40,10 @@ def _run_dense(x, W_g, W_u, W_d, stream=None):
     return y, ws
 
 
+# d = 4096 with T >= 128 selects 256-token tiles (one full tile and a 44-row tail at T = 300):
+# on CTA pairs at I = 512, on single CTAs at I = 384.
 @pytest.mark.parametrize("T,d,I", [(64, 128, 256), (1, 128, 256), (333, 2048, 1024),
-                                   (700, 384, 640)])
+                                   (700, 384, 640), (300, 4096, 512), (300, 4096, 384)])
 def test_dense_ffn_matches_oracle(T, d, I):
     x, W_g, W_u, W_d = _dense_case(T, d, I, seed=T + d)
     y, ws = _run_dense(x, W_g, W_u, W_d)
