@@ -1,6 +1,7 @@
 """Host-side tests (no GPU): the C-ABI library loads and exports every entry point the header
-declares, argument errors return the documented codes before any CUDA call, and the
-multi-process replica timing of bench.py reduces to the maximum over ranks (gloo, 2 ranks).
+declares, argument errors return the documented codes before any CUDA call, the
+multi-process replica timing of bench.py reduces to the maximum over ranks (gloo, 2 ranks), and
+the benchmark's algorithmic work model and GEMM source hash behave as its roofline needs.
 """
 import ctypes
 import os
@@ -159,3 +160,41 @@ def test_replica_timing_is_max_over_ranks_gloo():
     for rank, m, tput in res:
         assert m == 17.25
         assert tput == pytest.approx(2 * 16384 * 10 / 0.01725)
+
+
+def _bench():
+    import sys
+    if ROOT not in sys.path:
+        sys.path.insert(0, ROOT)
+    import bench
+    return bench
+
+
+def test_work_model_per_unit_figures():
+    # The roofline's algorithmic work, on a routing small enough to count by hand: T = 4 tokens,
+    # d = 8, I = 16, N = 3 FFN experts + Z = 1 zero expert, K = 2; counts 3, 0, 2 on the FFN
+    # experts (A = 5 slots, U = 2 experts used) and 3 on the zero expert.
+    from mixture_experts_layer_38_b200.workloads import Workload
+    w = Workload("hand", T=4, d=8, N=3, Z=1, K=2, I=16)
+    A, U, flops, nbytes = _bench().work_model(w, [3, 0, 2, 3])
+    assert (A, U) == (5, 2)
+    assert flops == {"router_gemm": 256, "ffn_up_gemm": 2560, "ffn_down_gemm": 1280}
+    assert nbytes == {"router_gemm": 192, "ffn_up_gemm": 1264, "ffn_down_gemm": 752,
+                      "dispatch": 160, "combine": 208}
+    _, _, _, nbytes8 = _bench().work_model(w, [3, 0, 2, 3], wb=1)  # E4M3 weight codes
+    assert nbytes8["ffn_up_gemm"] == 512 + 80 + 160 and nbytes8["ffn_down_gemm"] == 256 + 240
+
+
+def test_gemm_source_hash_ignores_comments_only():
+    # The recorded DRAM traffic is reported only while the GEMM sources hash to the captured
+    # version: comment edits must keep the hash, any code edit must change it.
+    bench = _bench()
+
+    def real(path):
+        with open(os.path.join(ROOT, path), encoding="utf-8") as f:
+            return f.read()
+    h0 = bench.gemm_source_hash()
+    assert bench.gemm_source_hash(real) == h0
+    assert bench.gemm_source_hash(lambda p: real(p) + "\n// note\n/* block\n note */\n") == h0
+    assert bench.gemm_source_hash(
+        lambda p: real(p).replace("constexpr int kBK = 64;", "constexpr int kBK = 32;")) != h0
