@@ -235,6 +235,159 @@ def work_model(w, counts, wb=2):
     return A, U, flops, bytes_
 
 
+def stage_durations(events):
+    """Per-stage milliseconds summed over the timed steps (events recorded by moe_forward_timed)."""
+    stage_ms = {n: 0.0 for n in mb.STAGE_NAMES}
+    for ev in events:
+        for si, n in enumerate(mb.STAGE_NAMES):
+            stage_ms[n] += ev[si].elapsed_time(ev[si + 1])
+    return stage_ms
+
+
+def step_work(w, hist, wb=2):
+    """Algorithmic FLOPs and bytes summed over the steps whose per-expert counts are `hist`."""
+    tot_flops = {k: 0 for k in ("router_gemm", "ffn_up_gemm", "ffn_down_gemm")}
+    tot_bytes = {k: 0 for k in ("router_gemm", "ffn_up_gemm", "ffn_down_gemm", "dispatch",
+                                "combine")}
+    A_steps, U_steps, load_ratio = [], [], []
+    for c in hist:
+        A, U, fl, by = work_model(w, c, wb=wb)
+        A_steps.append(A)
+        U_steps.append(U)
+        ffn = c[:w.N]
+        load_ratio.append(float(ffn.max()) / max(float(ffn.mean()), 1e-30))
+        for k in fl:
+            tot_flops[k] += fl[k]
+        for k in by:
+            tot_bytes[k] += by[k]
+    return tot_flops, tot_bytes, (A_steps, U_steps, load_ratio)
+
+
+def roofline_of(w, stage_ms, tot_flops, tot_bytes, fp8=False):
+    """Roofline record of the dominant (longest) stage: FLOP/s against the burst bf16 peak for
+    a contraction at prefill-like sizes, bytes/s against the HBM copy peak at decode."""
+    pk, pk_src = peaks()
+    kernel = max(stage_ms, key=stage_ms.get)
+    if w.name == "decode" or kernel not in tot_flops:
+        achieved = tot_bytes[kernel] / (stage_ms[kernel] / 1e3) / 1e9
+        peak = pk["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s"}
+        peak_name = "hbm_gbs"
+    else:
+        # The kernel is event-timed over a sub-second run of steps: the burst peak applies.
+        achieved = tot_flops[kernel] / (stage_ms[kernel] / 1e3) / 1e12
+        peak = pk["bf16_tflops"]
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                "unit": "TFLOP/s"}
+        peak_name = "bf16_tflops (burst)"
+        if "bf16_tflops_sustained" in pk:
+            roof["frac_of_sustained"] = round(achieved / pk["bf16_tflops_sustained"], 4)
+    roof["frac"] = round(achieved / peak, 4)
+    # the datasheet figures (dense bf16 2250 TFLOP/s, HBM3e 8000 GB/s), for context
+    roof["frac_of_nominal"] = round(achieved / (NOMINAL_HBM_GBS if roof["bound"] == "hbm"
+                                                else NOMINAL_BF16_TFLOPS), 4)
+    tr = NCU_TRAFFIC.get((w.name + ("+fp8" if fp8 else ""), kernel))
+    roof["traffic"] = tr["bytes_per_launch"] if tr and tr["src"] == gemm_source_hash() else None
+    roof["kernel"] = kernel
+    roof["peak_source"] = f"{pk_src} {peak_name}"
+    return roof
+
+
+def layer_of(flops, bytes_, ms, decode=False):
+    """The whole step against both rooflines, and the target the workload is held to: at
+    prefill-like sizes >= 0.60 of the bf16 peak, at decode >= 0.70 of HBM bandwidth."""
+    pk, _ = peaks()
+    tflops = flops / (ms / 1e3) / 1e12
+    gbs = bytes_ / (ms / 1e3) / 1e9
+    layer = {"tflops": round(tflops, 1),
+             "frac_of_bf16_peak": round(tflops / pk["bf16_tflops"], 4),
+             "frac_of_nominal_bf16": round(tflops / NOMINAL_BF16_TFLOPS, 4),
+             "gbs": round(gbs, 1),
+             "frac_of_hbm_peak": round(gbs / pk["hbm_gbs"], 4),
+             "frac_of_nominal_hbm": round(gbs / NOMINAL_HBM_GBS, 4)}
+    if decode:
+        layer["target"] = {"what": "whole step >= 0.70 of measured HBM bandwidth",
+                           "frac": layer["frac_of_hbm_peak"],
+                           "met": layer["frac_of_hbm_peak"] >= 0.70}
+    else:
+        layer["target"] = {"what": "whole step >= 0.60 of measured burst bf16 peak",
+                           "frac": layer["frac_of_bf16_peak"],
+                           "met": layer["frac_of_bf16_peak"] >= 0.60}
+    return layer
+
+
+def near_tie_tokens(dm, x, W_r, b, ws):
+    """Tokens whose K-th vs (K+1)-th biased-score gap (the GPU's fp32 gap from moe_route) is at
+    most 1e-4 on the bench's x with the current biases: where the routing rule allows any
+    eps-valid set instead of one bit-exact set."""
+    idx = torch.empty((dm.T, dm.K), dtype=torch.int32, device=x.device)
+    gate = torch.empty((dm.T, dm.K), dtype=torch.float32, device=x.device)
+    gap = torch.empty((dm.T,), dtype=torch.float32, device=x.device)
+    mb.moe_route(dm, x, W_r, b, idx, gate, gap, ws)
+    return int((gap <= 1e-4).sum().item())
+
+
+def decode_record(args, wt, device, rank, world):
+    """The decode workload (T = 128) timed on the given expert weights, as its own record:
+    ms per step, tokens/s, the dominant kernel against the HBM peak, the whole step's
+    fractions, per-stage times and clocks.  Every rank runs it (the max over ranks is taken)."""
+    w = WORKLOADS["decode"]
+    x = make_tokens(w, device, seed=args.seed + rank)
+    dm = mb.dims(w.T, w.d, w.N, w.Z, w.K, w.I)
+    ws = mb.alloc_workspace(dm, device)
+    y = torch.empty((w.T, w.d), dtype=torch.bfloat16, device=device)
+    b = wt["b"].clone()
+    pid_state = torch.zeros(2, dtype=torch.float32, device=device)
+    params = mb.PidParams(w.pid_target, *PID_GAINS, 0.0)
+    steps = max(args.steps, 60)  # ~0.1 s: enough clock samples
+    counts = torch.zeros((args.warmup + steps, w.E), dtype=torch.int32, device=device)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(mb.NUM_STAGE_EVENTS)]
+              for _ in range(steps)]
+    stream = torch.cuda.current_stream()
+    for ev in events:
+        for e in ev:
+            e.record(stream)
+    for i in range(args.warmup):
+        mb.moe_forward(dm, x, wt["W_r"], b, wt["W_g"], wt["W_u"], wt["W_d"], y, counts[i], ws)
+        mb.moe_bias_update(dm, counts[i], b, pid_state, params)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = ClockSampler(device)
+    clocks.start()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(steps):
+        c = counts[args.warmup + i]
+        mb.moe_forward_timed(dm, x, wt["W_r"], b, wt["W_g"], wt["W_u"], wt["W_d"], y, c, ws,
+                             events[i])
+        mb.moe_bias_update(dm, c, b, pid_state, params)
+    end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = max_over_ranks(start.elapsed_time(end), world, device)
+    status = mb.moe_last_device_error(ws)
+    if status != 0:
+        raise RuntimeError(f"device status {status:#x} after the decode steps")
+    stage_ms = stage_durations(events)
+    tot_flops, tot_bytes, (A_steps, U_steps, _) = step_work(
+        w, counts[args.warmup:].cpu().numpy())
+    layer = layer_of(sum(tot_flops.values()), sum(tot_bytes.values()), ms, decode=True)
+    return {
+        "workload": w.name, "T": w.T, "steps": steps,
+        "ms_per_step": round(ms / steps, 4),
+        "value": round(job_throughput(world, w.T, steps, ms), 1), "unit": UNIT,
+        "roofline": roofline_of(w, stage_ms, tot_flops, tot_bytes),
+        "layer": layer,
+        "stages_ms": {k: round(v / steps, 4) for k, v in stage_ms.items()},
+        "mean_ffn_experts_per_token": round(float(np.mean(A_steps)) / w.T, 4),
+        "distinct_ffn_experts": int(np.mean(U_steps)),
+        "near_tie_tokens": near_tie_tokens(dm, x, wt["W_r"], b, ws),
+        "clocks": clk,
+        "gpu_launches": LAUNCHES_PER_STEP * steps,
+    }
+
+
 # ------------------------------------------------------------------------------ CPU oracle
 def oracle_tokens_per_s(w, x_dev, wt, b, n_tokens, seed, cache=None):
     """The oracle, as it stands, on a seeded sample of tokens; weight fetches not timed."""
@@ -387,61 +540,20 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError(f"device status {status:#x} after the timed steps")
 
     # per-stage durations and algorithmic work of the timed steps
-    stage_ms = {n: 0.0 for n in mb.STAGE_NAMES}
-    for ev in events:
-        for si, n in enumerate(mb.STAGE_NAMES):
-            stage_ms[n] += ev[si].elapsed_time(ev[si + 1])
+    stage_ms = stage_durations(events)
     hist = counts[args.warmup:n_steps].cpu().numpy()
-    tot_flops = {k: 0 for k in ("router_gemm", "ffn_up_gemm", "ffn_down_gemm")}
-    tot_bytes = {k: 0 for k in ("router_gemm", "ffn_up_gemm", "ffn_down_gemm", "dispatch",
-                                "combine")}
-    A_steps, U_steps, load_ratio = [], [], []
-    for c in hist:
-        A, U, fl, by = work_model(w, c, wb=1 if args.fp8 else 2)
-        A_steps.append(A)
-        U_steps.append(U)
-        ffn = c[:w.N]
-        load_ratio.append(float(ffn.max()) / max(float(ffn.mean()), 1e-30))
-        for k in fl:
-            tot_flops[k] += fl[k]
-        for k in by:
-            tot_bytes[k] += by[k]
-    pk, pk_src = peaks()
-    dominant = max(stage_ms, key=stage_ms.get)
-    hbm_bound = w.name == "decode"
-    kernel = dominant
-    if hbm_bound or kernel not in tot_flops:
-        achieved = tot_bytes[kernel] / (stage_ms[kernel] / 1e3) / 1e9
-        peak = pk["hbm_gbs"]
-        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s"}
-        peak_name = "hbm_gbs"
-    else:
-        achieved = tot_flops[kernel] / (stage_ms[kernel] / 1e3) / 1e12
-        peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
-        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
-                "unit": "TFLOP/s"}
-        peak_name = "bf16_tflops_sustained"
-    roof["frac"] = round(achieved / peak, 4)
-    # the datasheet figures (dense bf16 2250 TFLOP/s, HBM3e 8000 GB/s), for context
-    roof["frac_of_nominal"] = round(achieved / (NOMINAL_HBM_GBS if roof["bound"] == "hbm"
-                                                else NOMINAL_BF16_TFLOPS), 4)
-    tr = NCU_TRAFFIC.get((w.name + ("+fp8" if args.fp8 else ""), kernel))
-    roof["traffic"] = tr["bytes_per_launch"] if tr and tr["src"] == gemm_source_hash() else None
-    roof["kernel"] = kernel
-    roof["peak_source"] = f"{pk_src} {peak_name}"
+    tot_flops, tot_bytes, routing = step_work(w, hist, wb=1 if args.fp8 else 2)
+    roof = roofline_of(w, stage_ms, tot_flops, tot_bytes, fp8=args.fp8)
     layer_flops = sum(tot_flops.values())
     if scmoe is not None:
         scmoe["step_ms"] = round(ms / args.steps, 4)
         layer_flops += scmoe["dense_flop_per_step"] * args.steps
-    layer_tflops = layer_flops / (ms / 1e3) / 1e12
-    layer_gbs = sum(tot_bytes.values()) / (ms / 1e3) / 1e9
-    routing = (A_steps, U_steps, load_ratio)
-    layer = {"tflops": round(layer_tflops, 1),
-             "frac_of_bf16_peak": round(layer_tflops / pk["bf16_tflops"], 4),
-             "frac_of_nominal_bf16": round(layer_tflops / NOMINAL_BF16_TFLOPS, 4),
-             "gbs": round(layer_gbs, 1),
-             "frac_of_hbm_peak": round(layer_gbs / pk["hbm_gbs"], 4),
-             "frac_of_nominal_hbm": round(layer_gbs / NOMINAL_HBM_GBS, 4)}
+    layer = layer_of(layer_flops, sum(tot_bytes.values()), ms, decode=w.name == "decode")
+    layer["near_tie_tokens"] = near_tie_tokens(dm, x, wt["W_r"], b, ws)
+    if not args.no_decode and w.name != "decode" and w.d == WORKLOADS["decode"].d and \
+            w.N == WORKLOADS["decode"].N and w.I == WORKLOADS["decode"].I and not args.fp8:
+        # The second target's workload on the same expert weights (decode shares every one).
+        layer["decode"] = decode_record(args, wt, device, rank, world)
     if scmoe is not None:
         layer["scmoe"] = scmoe
 
@@ -514,6 +626,8 @@ def run_ours(args, rank, world, local_rank):
 
 def finish(args, w, world, rank, ms_max, routing, roof, layer, stage_ms, clk, e2e, x, wt, b):
     A_steps, U_steps, load_ratio = routing
+    near_ties = layer.pop("near_tie_tokens", None)
+    decode = layer.pop("decode", None)
     result = {
         "metric": METRIC, "value": round(job_throughput(world, w.T, args.steps, ms_max), 1),
         "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -537,11 +651,14 @@ def finish(args, w, world, rank, ms_max, routing, roof, layer, stage_ms, clk, e2
         },
         "roofline": roof,
         "layer": layer,
+        "near_tie_tokens": near_ties,
         "stages_ms": {k: round(v / args.steps, 4) for k, v in stage_ms.items()},
         "clocks": clk,
         "e2e": e2e,
         "gpu_launches": (LAUNCHES_PER_STEP + (2 if args.scmoe else 0)) * args.steps,
     }
+    if decode is not None:
+        result["decode"] = decode
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         n = args.cpu_sample or default_sample(w)
         log(f"oracle CPU baseline on {n} sampled tokens ...")
@@ -606,6 +723,8 @@ def main():
     ap.add_argument("--cpu-sample", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg (profiling)")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="skip the decode (T=128) record on the same weights")
     ap.add_argument("--renormalize-gates", action="store_true",
                     help="variant: gates renormalised over the K selected experts")
     ap.add_argument("--scmoe", type=int, default=0, metavar="I_DENSE",

@@ -119,6 +119,16 @@ int moe_route(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *W_r, cons
               int32_t *topk_idx, float *topk_gate, float *gap, void *ws, size_t ws_bytes,
               void *stream);
 
+/* The router logits l = x W_r^T (same section: the scores the softmax router R normalises)
+ * that the last moe_route or moe_forward with these dims computed into workspace `ws`, summed
+ * over the router GEMM's split-K partials in the same fixed order the top-K kernel sums them,
+ * so they are bit-identical to the logits the selection used.  For inspecting the router's
+ * fp32 accuracy; calls on the same stream after that routing call see its logits.
+ *   ws      the workspace given to that call (>= moe_scratch_size(dims) bytes)
+ *   logits  [T, N+Z] fp32 (out) */
+int moe_router_logits(const moe_dims *dims, const void *ws, size_t ws_bytes, float *logits,
+                      void *stream);
+
 /* Dispatch: group the FFN slots by expert (zero-expert slots are never copied).  Stable
  * counting sort with key (expert id, token), deterministic.
  *   x         [T, d] bf16, topk_idx/topk_gate [T, K] as produced by moe_route (ids in
@@ -198,10 +208,13 @@ int moe_dense_ffn(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *W_g,
  * + (sum of the zero-expert gates of t) * x_t, accumulated in fp32 in that fixed order and
  * rounded once to bf16.  Zero experts are identities ("衝上熱搜！美團大模型，靠「快」火了",
  * §零計算專家), so they cost one fused scalar-times-row term and no copy.
- *   y [T, d] bf16 (out). */
+ *   y  [T, d] bf16 (out).
+ *   ws a workspace of at least 256 bytes whose status word (its first 4 bytes, zero before the
+ *      first call) records MOE_DEV_BAD_ROWS when an FFN slot's slot_pos lies outside
+ *      [0, T*K); that slot's term is skipped.  Any workspace of the other calls will do. */
 int moe_combine(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *y_perm,
                 const int32_t *topk_idx, const float *topk_gate, const int32_t *slot_pos,
-                moe_bf16 *y, void *stream);
+                moe_bf16 *y, void *ws, size_t ws_bytes, void *stream);
 
 /* PID update of the FFN experts' biases from one batch's counts (same page and section, last
  * paragraph; the law is a reading, the pages give no equation):
@@ -281,6 +294,15 @@ int moe_forward_fp8(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *W_r
 /* Synchronises `stream`, returns the device status word of the workspace (MOE_DEV_* code,
  * 0 if none) and clears it.  Returns a negative value if the synchronisation itself failed. */
 int moe_last_device_error(void *ws, void *stream);
+
+/* Testing hook for the failure path of the grouped GEMMs (moe_route's router GEMM, the expert
+ * FFN GEMMs, moe_dense_ffn): sets, for launches enqueued afterwards by this process, the SM
+ * clock cycles after which one pipeline wait gives up; 0 restores the default of 2^32 cycles.
+ * With a limit shorter than a real wait (e.g. 64 cycles: no tile completes that fast) the
+ * kernel records MOE_DEV_WAIT_TIMEOUT, unwinds every role, waits (bounded) for its copies and
+ * MMAs in flight, frees its tensor memory and exits, so the context stays usable.  Not for
+ * production use.  Returns MOE_ERR_ARG for a negative value. */
+int moe_debug_set_wait_limit(int64_t cycles);
 
 #ifdef __cplusplus
 }

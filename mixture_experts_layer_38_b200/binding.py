@@ -20,6 +20,7 @@ EXPORTS = (
     "moe_expert_ffn", "moe_combine", "moe_bias_update", "moe_forward", "moe_forward_timed",
     "moe_last_device_error", "moe_dispatch_noalloc", "moe_expert_ffn_gather",
     "moe_quantize_fp8", "moe_expert_ffn_fp8", "moe_forward_fp8", "moe_dense_ffn",
+    "moe_router_logits", "moe_debug_set_wait_limit",
 )
 NUM_STAGE_EVENTS = 7
 STAGE_NAMES = ("router_gemm", "route_topk", "dispatch", "ffn_up_gemm", "ffn_down_gemm",
@@ -74,7 +75,9 @@ def lib():
         L.moe_route.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, _S, _P]
         L.moe_dispatch.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]
         L.moe_expert_ffn.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]
-        L.moe_combine.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P]
+        L.moe_combine.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, _S, _P]
+        L.moe_router_logits.argtypes = [_DP, _P, _S, _P, _P]
+        L.moe_debug_set_wait_limit.argtypes = [ctypes.c_int64]
         L.moe_bias_update.argtypes = [_DP, _P, _P, _P, ctypes.POINTER(PidParams), _P]
         L.moe_forward.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]
         L.moe_forward_timed.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S,
@@ -92,7 +95,7 @@ def lib():
                   "moe_bias_update", "moe_forward", "moe_forward_timed",
                   "moe_last_device_error", "moe_dispatch_noalloc", "moe_expert_ffn_gather",
                   "moe_quantize_fp8", "moe_expert_ffn_fp8", "moe_forward_fp8",
-                  "moe_dense_ffn"):
+                  "moe_dense_ffn", "moe_router_logits", "moe_debug_set_wait_limit"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -197,7 +200,7 @@ def moe_dispatch_noalloc(dm, x, topk_idx, topk_gate, counts, offsets, perm_tok, 
         _ptr(counts, torch.int32, (E,), "counts"), _ptr(offsets, torch.int32, (dm.N + 1,), "offsets"),
         _ptr(perm_tok, torch.int32, (R,), "perm_tok"), _ptr(perm_gate, torch.float32, (R,), "perm_gate"),
         _ptr(slot_pos, torch.int32, (dm.T, dm.K), "slot_pos"),
-        _ptr(x_perm, torch.bfloat16, (R, dm.d), "x_perm"), _stream(stream))
+        _ptr(x_perm, torch.bfloat16, (R, dm.d), "x_perm", nullable=True), _stream(stream))
     _check("moe_dispatch_noalloc", rc)
 
 
@@ -233,16 +236,31 @@ def moe_expert_ffn_gather(dm, x, perm_tok, offsets, perm_gate, W_g, W_u, W_d, h,
     _check("moe_expert_ffn_gather", rc)
 
 
-def moe_combine(dm, x, y_perm, topk_idx, topk_gate, slot_pos, y, stream=None):
+def moe_combine(dm, x, y_perm, topk_idx, topk_gate, slot_pos, y, ws, stream=None):
     R = dm.T * dm.K
+    w, n = _ws(ws)
     rc = lib().moe_combine(
         ctypes.byref(dm), _ptr(x, torch.bfloat16, (dm.T, dm.d), "x"),
         _ptr(y_perm, torch.bfloat16, (R, dm.d), "y_perm"),
         _ptr(topk_idx, torch.int32, (dm.T, dm.K), "topk_idx"),
         _ptr(topk_gate, torch.float32, (dm.T, dm.K), "topk_gate"),
         _ptr(slot_pos, torch.int32, (dm.T, dm.K), "slot_pos"),
-        _ptr(y, torch.bfloat16, (dm.T, dm.d), "y"), _stream(stream))
+        _ptr(y, torch.bfloat16, (dm.T, dm.d), "y"), w, n, _stream(stream))
     _check("moe_combine", rc)
+
+
+def moe_router_logits(dm, ws, logits, stream=None):
+    """The fp32 router logits [T, N+Z] of the last routing call on ``ws`` (same dims)."""
+    w, n = _ws(ws)
+    rc = lib().moe_router_logits(
+        ctypes.byref(dm), w, n, _ptr(logits, torch.float32, (dm.T, dm.N + dm.Z), "logits"),
+        _stream(stream))
+    _check("moe_router_logits", rc)
+
+
+def moe_debug_set_wait_limit(cycles: int):
+    """Testing hook: the grouped GEMMs' per-wait limit in SM cycles (0 = the default)."""
+    _check("moe_debug_set_wait_limit", lib().moe_debug_set_wait_limit(int(cycles)))
 
 
 def moe_bias_update(dm, counts, b, pid_state, params: PidParams, stream=None):

@@ -56,16 +56,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return done != 0;
 }
 
-// Waits until the phase with the given parity has completed.  Gives up after
-// kWaitLimitCycles, or as soon as *abort becomes non-zero, and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
-                                          volatile int *abort) {
+// Waits until the phase with the given parity has completed.  Gives up after `limit` cycles
+// (kWaitLimitCycles unless a test shortens it), or as soon as *abort becomes non-zero, and
+// returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                          long long limit = kWaitLimitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (clock64() - t0 > kWaitLimitCycles) return false;
+    if (clock64() - t0 > limit) return false;
   }
 }
 

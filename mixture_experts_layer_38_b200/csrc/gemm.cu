@@ -41,6 +41,8 @@
 // roles unwind, in-flight copies and MMAs are drained (again bounded) and TMEM is freed.
 #include <cuda_fp8.h>
 
+#include <atomic>
+
 #include "device.cuh"
 #include "kernels.cuh"
 
@@ -119,11 +121,16 @@ struct Tile {
   int split;
 };
 
-// Token tiles of a group (expert) with c rows: floor(c/128) full 128-row tiles ("heavy":
-// compute-bound at d = 6144) and, if c % 128 != 0, one partial tail tile ("light": for the many
+// Token tiles of a group (expert) with c rows: floor(c/BN) full BN-row tiles ("heavy":
+// compute-bound at d = 6144) and, if c % BN != 0, one partial tail tile ("light": for the many
 // experts with a handful of tokens it only streams the expert's weights).  The schedule merges
 // the two lists so the tiles in flight at any moment mix both kinds and the tensor cores and
 // HBM are busy together: of the first p+1 merged positions, floor((p+1) L / (H+L)) are light.
+// Work items (token tile, weight tile, split) are dealt round-robin to the persistent units
+// (CTAs, or CTA pairs).  Every SM therefore streams some of the time: one SM keeps only ~128 KB
+// of weights in flight, about 45-60 GB/s, so HBM needs most SMs streaming at once (measured:
+// dedicating a subset of units to the tail tiles and the rest to full tiles was slower for
+// every split tried, the tail side never reaching the bandwidth the interleaving gets).
 struct Schedule {
   const int *hpre;  // [G + 1] prefix of full tiles per group (shared memory)
   const int *lpre;  // [G + 1] prefix of tail tiles per group
@@ -131,7 +138,7 @@ struct Schedule {
   int H, L;         // total full / tail tiles
   int m_tiles;
   int splits;
-  int total;
+  int total;        // work items
 };
 
 __device__ __forceinline__ int group_off(const GemmArgs &a, int g) {
@@ -266,9 +273,10 @@ __device__ __forceinline__ int m_tiles_of(int M) {
 }
 
 // Bounded wait by lane 0 of a warp, result broadcast so the warp stays converged.
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                          long long limit) {
   int ok = 0;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort) ? 1 : 0;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, limit) ? 1 : 0;
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
@@ -473,6 +481,7 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER, PR>::kThreads, 1)
   sched.m_tiles = m_tiles_of<EPI, PR>(args.M);
   sched.splits = EPI == kEpiF32 ? args.k_splits : 1;
   sched.total = sched.total * sched.m_tiles * sched.splits;
+  const long long wlim = args.wait_limit > 0 ? args.wait_limit : kWaitLimitCycles;
   tc_fence_before();
   if (PR) cluster_sync();  // both CTAs' barriers initialised before any remote arrival
   else __syncthreads();
@@ -501,7 +510,7 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER, PR>::kThreads, 1)
                                         (GATHER ? 0 : t.nb * kBK * 2);
         const uint64_t pol_w = t.once ? pol_w_once : pol_w_reused;
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
-          if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag)) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, wlim)) {
             signal_abort(args, abort_flag);
             ok = false;
             break;
@@ -595,7 +604,7 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER, PR>::kThreads, 1)
         const Tile t = decode_tile<EPI, BN, PR>(args, sched, tile, rank);
         const int buf = it % C::kAccBufs;
         const uint32_t use = (uint32_t)(it / C::kAccBufs);
-        if (!mbar_wait(&tempty_bar[buf], (use & 1) ^ 1, abort_flag)) {
+        if (!mbar_wait(&tempty_bar[buf], (use & 1) ^ 1, abort_flag, wlim)) {
           signal_abort(args, abort_flag);
           ok = false;
           break;
@@ -605,8 +614,8 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER, PR>::kThreads, 1)
         const uint32_t d1 = d0 + BN;
         const uint32_t idesc = idesc_bf16_f32(PR ? 2 * kBM : kBM, t.nb);
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
-          if (!mbar_wait(&full_bar[stage], phase, abort_flag) ||
-              (WQ && !mbar_wait(&cfull_bar[cslot], cphase, abort_flag))) {
+          if (!mbar_wait(&full_bar[stage], phase, abort_flag, wlim) ||
+              (WQ && !mbar_wait(&cfull_bar[cslot], cphase, abort_flag, wlim))) {
             signal_abort(args, abort_flag);
             ok = false;
             break;
@@ -676,7 +685,7 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER, PR>::kThreads, 1)
         rix[i] = v;
       }
       for (int kb = t.kb0; kb < t.kb1; ++kb) {
-        if (!warp_wait(&empty_bar[stage], phase ^ 1, abort_flag)) {
+        if (!warp_wait(&empty_bar[stage], phase ^ 1, abort_flag, wlim)) {
           if (lane == 0) signal_abort(args, abort_flag);
           ok = false;
           break;
@@ -706,8 +715,8 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER, PR>::kThreads, 1)
       const float *scales = (half ? args.scale_a1 : args.scale_a0) + (row / 128) * args.scale_ld;
       const bool mine = half == 0 || t.has_a1;
       for (int kb = t.kb0; kb < t.kb1; ++kb) {
-        if (!warp_wait(&full_bar[stage], phase, abort_flag) ||
-            !warp_wait(&cempty_bar[cslot], cphase ^ 1, abort_flag)) {
+        if (!warp_wait(&full_bar[stage], phase, abort_flag, wlim) ||
+            !warp_wait(&cempty_bar[cslot], cphase ^ 1, abort_flag, wlim)) {
           if (lane == 0) signal_abort(args, abort_flag);
           ok = false;
           break;
@@ -737,7 +746,7 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER, PR>::kThreads, 1)
       const Tile t = decode_tile<EPI, BN, PR>(args, sched, tile, rank);
       const int buf = it % C::kAccBufs;
       const uint32_t use = (uint32_t)(it / C::kAccBufs);
-      if (!warp_wait(&tfull_bar[buf], use & 1, abort_flag)) {
+      if (!warp_wait(&tfull_bar[buf], use & 1, abort_flag, wlim)) {
         if (lane == 0) signal_abort(args, abort_flag);
         break;
       }
@@ -776,6 +785,15 @@ cudaError_t set_smem_limit() {
                               Cfg<BN, WQ, GATHER, PR>::kSmemBytes);
 }
 
+// Wait limit applied to launches (0: kWaitLimitCycles); only the timeout-path tests change it.
+std::atomic<long long> g_wait_limit{0};
+
+GemmArgs with_limit(const GemmArgs &args) {
+  GemmArgs a = args;
+  a.wait_limit = g_wait_limit.load(std::memory_order_relaxed);
+  return a;
+}
+
 using PairCfg = Cfg<256, false, false, true>;
 constexpr int kMaxDevices = 64;
 int g_max_pairs[kMaxDevices] = {0};
@@ -812,7 +830,8 @@ cudaError_t prepare_pair(int device) {
 }
 
 template <int BN>
-cudaError_t launch_bn(int epi, const GemmArgs &args, int grid, cudaStream_t stream) {
+cudaError_t launch_bn(int epi, const GemmArgs &args_in, int grid, cudaStream_t stream) {
+  const GemmArgs args = with_limit(args_in);
   constexpr int smem = Cfg<BN>::kSmemBytes;
   constexpr int threads = Cfg<BN>::kThreads;
   switch (epi) {
@@ -852,6 +871,10 @@ cudaError_t gemm_prepare(int device) {
   return set_smem_limit<kEpiF32, 256>();
 }
 
+void gemm_set_wait_limit(long long cycles) {
+  g_wait_limit.store(cycles > 0 ? cycles : 0, std::memory_order_relaxed);
+}
+
 int gemm_tile_tokens(long long rows, int groups, int K) {
   // 256-token tiles need enough rows per group to fill them (mean rows per group, an upper
   // bound since zero-expert slots are counted too) and a long reduction, over which the
@@ -863,9 +886,10 @@ int gemm_max_pairs(int device) {
   return (device >= 0 && device < kMaxDevices) ? g_max_pairs[device] : 0;
 }
 
-cudaError_t launch_grouped_gemm_pair(int epi, const GemmArgs &args, int pairs,
+cudaError_t launch_grouped_gemm_pair(int epi, const GemmArgs &args_in, int pairs,
                                      cudaStream_t stream) {
   if (pairs <= 0) return cudaErrorInvalidConfiguration;
+  const GemmArgs args = with_limit(args_in);
   cudaLaunchAttribute attr[1];
   const cudaLaunchConfig_t cfg = pair_config(pairs, stream, attr);
   switch (epi) {
@@ -886,9 +910,10 @@ cudaError_t launch_grouped_gemm(int epi, const GemmArgs &args, int grid, int til
                             : launch_bn<128>(epi, args, grid, stream);
 }
 
-cudaError_t launch_grouped_gemm_fp8(int epi, const GemmArgs &args, int grid,
+cudaError_t launch_grouped_gemm_fp8(int epi, const GemmArgs &args_in, int grid,
                                     cudaStream_t stream) {
   using C = Cfg<128, true>;
+  const GemmArgs args = with_limit(args_in);
   if (epi == kEpiSwiGLU)
     grouped_gemm_kernel<kEpiSwiGLU, 128, true, false>
         <<<grid, C::kThreads, C::kSmemBytes, stream>>>(args);

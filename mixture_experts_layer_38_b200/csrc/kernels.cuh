@@ -46,6 +46,9 @@ struct GemmArgs {
   const float *scale_a0;
   const float *scale_a1;
   int scale_ld;
+  // Cycles after which one pipeline wait gives up (set by the launchers; see
+  // gemm_set_wait_limit).
+  long long wait_limit;
 };
 
 // Grouped GEMM block: warp 0 issues TMA loads, warp 1 allocates TMEM and issues MMAs, and
@@ -55,6 +58,9 @@ struct GemmArgs {
 constexpr int kGemmEpiWarps = 4;
 constexpr int kGemmThreads = 64 + 32 * kGemmEpiWarps;
 cudaError_t gemm_prepare(int device);  // sets the kernels' shared-memory limit once per device
+// Wait limit in SM cycles for grouped-GEMM launches enqueued from now on (0: the default,
+// kWaitLimitCycles).  A testing hook for the timeout path.
+void gemm_set_wait_limit(long long cycles);
 // Token-tile width (128 or 256) for `rows` activation rows over `groups` groups, reduction K.
 int gemm_tile_tokens(long long rows, int groups, int K);
 cudaError_t launch_grouped_gemm(int epi, const GemmArgs &args, int grid, int tile_tokens,
@@ -80,6 +86,10 @@ cudaError_t launch_quantize_fp8(const uint16_t *w, long long G, long long R, lon
 cudaError_t launch_route_topk(const float *logits, int splits, int T, int E, int K,
                               const float *b, bool renormalize, int32_t *topk_idx,
                               float *topk_gate, float *gap, int *status, cudaStream_t stream);
+
+// logits [splits][T][ld] fp32 partials -> l [T][E] fp32, summed in the top-K kernels' order.
+cudaError_t launch_router_logits(const float *partial, int splits, int T, int E, float *out,
+                                 int num_sms, cudaStream_t stream);
 
 // ------------------------------------------------------------------ dispatch
 constexpr int kDispatchChunk = 256;  // tokens per histogram chunk (8 warps x 32)

@@ -560,7 +560,7 @@ int moe_dense_ffn(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *W_g,
 
 int moe_combine(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *y_perm,
                 const int32_t *topk_idx, const float *topk_gate, const int32_t *slot_pos,
-                moe_bf16 *y, void *stream) {
+                moe_bf16 *y, void *ws, size_t ws_bytes, void *stream) {
   MOE_REQUIRE(dims != nullptr, MOE_ERR_ARG);
   MOE_REQUIRE(dims_ok(dims), MOE_ERR_SHAPE);
   MOE_CHECK_TOKEN_PTR(x, dims->T);
@@ -569,12 +569,36 @@ int moe_combine(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *y_perm,
   MOE_CHECK_TOKEN_PTR(topk_gate, dims->T);
   MOE_CHECK_TOKEN_PTR(slot_pos, dims->T);
   MOE_CHECK_TOKEN_PTR(y, dims->T);
+  int rc = check_ws(ws, ws_bytes, kAlign);  // the status word only
+  if (rc != MOE_OK) return rc;
   const DeviceInfo *di = nullptr;
-  const int rc = device_info(&di);
+  rc = device_info(&di);
   if (rc != MOE_OK) return rc;
   return to_status(launch_combine(x, y_perm, topk_idx, topk_gate, slot_pos, dims->T, dims->d,
-                                  dims->N, dims->K, dims->T * dims->K, y, nullptr,
+                                  dims->N, dims->K, dims->T * dims->K, y, at<int>(ws, 0),
                                   static_cast<cudaStream_t>(stream)));
+}
+
+int moe_router_logits(const moe_dims *dims, const void *ws, size_t ws_bytes, float *logits,
+                      void *stream) {
+  MOE_REQUIRE(dims != nullptr, MOE_ERR_ARG);
+  MOE_REQUIRE(dims_ok(dims), MOE_ERR_SHAPE);
+  MOE_CHECK_TOKEN_PTR(logits, dims->T);
+  const Layout L = layout_of(*dims);
+  int rc = check_ws(ws, ws_bytes, L.scratch_end);
+  if (rc != MOE_OK) return rc;
+  const DeviceInfo *di = nullptr;
+  rc = device_info(&di);
+  if (rc != MOE_OK) return rc;
+  return to_status(launch_router_logits(at<float>(const_cast<void *>(ws), L.logits), L.splits,
+                                        dims->T, dims->N + dims->Z, logits, di->sms,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+int moe_debug_set_wait_limit(int64_t cycles) {
+  MOE_REQUIRE(cycles >= 0, MOE_ERR_ARG);
+  gemm_set_wait_limit((long long)cycles);
+  return MOE_OK;
 }
 
 int moe_bias_update(const moe_dims *dims, const int32_t *counts, float *b, float *pid_state,

@@ -90,11 +90,13 @@ extern "C" int moe_dispatch_noalloc(const moe_dims *dims, const moe_bf16 *x,
   if (dims == nullptr) return MOE_ERR_ARG;
   if (moe_scratch_size(dims) == 0) return MOE_ERR_SHAPE;  // same limits as every entry point
   const int T = dims->T;
-  const void *token_bufs[] = {x, topk_idx, topk_gate, perm_tok, perm_gate, slot_pos, x_perm};
+  const void *token_bufs[] = {x, topk_idx, topk_gate, perm_tok, perm_gate, slot_pos};
   for (const void *p : token_bufs) {
     if (T > 0 && p == nullptr) return MOE_ERR_ARG;
     if (p != nullptr && !ok16(p)) return MOE_ERR_ALIGN;
   }
+  // As in moe_dispatch, a NULL x_perm skips the row copy (for moe_expert_ffn_gather).
+  if (x_perm != nullptr && !ok16(x_perm)) return MOE_ERR_ALIGN;
   if (counts == nullptr || offsets == nullptr) return MOE_ERR_ARG;
   if (!ok16(counts) || !ok16(offsets)) return MOE_ERR_ALIGN;
   const int E = dims->N + dims->Z;

@@ -15,6 +15,8 @@
 // thread timing.
 #include <math.h>
 
+#include <algorithm>
+
 #include "device.cuh"
 #include "kernels.cuh"
 
@@ -266,6 +268,31 @@ __global__ void __launch_bounds__(256)
 }
 
 }  // namespace
+
+// l[t, e] = sum of the split-K partial logits in split order, the same fixed order as the
+// top-K kernels above, so the result is bit-identical to the logits they select from.
+__global__ void __launch_bounds__(256)
+    router_logits_kernel(const float *__restrict__ partial, int splits, int T, int E, int ld,
+                         float *__restrict__ out) {
+  const long long n = (long long)T * E;
+  const long long split_stride = (long long)T * ld;
+  for (long long i = blockIdx.x * 256ll + threadIdx.x; i < n; i += (long long)gridDim.x * 256) {
+    const int t = (int)(i / E), e = (int)(i % E);
+    const float *src = partial + (long long)t * ld + e;
+    float v = src[0];
+    for (int sp = 1; sp < splits; ++sp) v += src[sp * split_stride];
+    out[i] = v;
+  }
+}
+
+cudaError_t launch_router_logits(const float *partial, int splits, int T, int E, float *out,
+                                 int num_sms, cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  const long long n = (long long)T * E;
+  const long long blocks = std::min<long long>((n + 255) / 256, 8ll * num_sms);
+  router_logits_kernel<<<(int)blocks, 256, 0, stream>>>(partial, splits, T, E, (E + 3) & ~3, out);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_route_topk(const float *logits, int splits, int T, int E, int K,
                               const float *b, bool renormalize, int32_t *topk_idx,

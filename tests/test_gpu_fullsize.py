@@ -1,8 +1,15 @@
 """GPU parity at the full 512 + 256-expert size (d = 6144, I = 2048, K = 12), in the launch
-configuration the benchmark times (moe_forward), on sampled tokens the oracle computes one by
-one, plus properties that hold for every token: counts sum to T*K, the dispatch is exactly
-the stable (expert, token) sort of the GPU's own routing, the staged calls reproduce
-moe_forward bit for bit, and the PID run of the skewed workload settles at its set-point.
+configuration the benchmark times (moe_forward).
+
+For EVERY token of each batch (decode 128, prefill 16384, skewed 8192): the routing against the
+oracle's router run on the whole batch (ids bit-exact wherever the oracle's gap exceeds 1e-4,
+near-ties counted and eps-valid, every gate equal to the oracle's probability of the id chosen
+up to the propagated error of the GPU's fp32 router logits, themselves within the fp32
+accumulation bound), and the dispatch tables bit-exact against the oracle's dispatch of the
+GPU's routing.  The layer output y on a seeded token sample plus the tokens the GPU routed
+differently from the oracle (near-ties), against the oracle's layer run on the GPU's routing.
+Besides: the staged calls reproduce moe_forward bit for bit, and the PID run of the skewed
+workload settles at its set-point.
 
 One weight set (38.7 GB, seed 0) serves decode, prefill and skewed: the three share every
 expert weight and differ only in column 0 of W_r for the skewed (Zipf) workload.
@@ -15,7 +22,9 @@ import oracle
 from mixture_experts_layer_38_b200 import binding as mb
 from mixture_experts_layer_38_b200.workloads import (WORKLOADS, apply_zipf_router, make_tokens,
                                                      make_weights)
-from parity import Stages, assert_y_close, check_dispatch_properties, check_routing, to_np
+from parity import (Stages, assert_y_close, check_dispatch_vs_oracle,
+                    check_gates_against_logits, check_routing_full, exact_logits,
+                    gpu_routing_for_oracle, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -34,7 +43,7 @@ def _fetch(wt):
     return lambda e: (wt["W_g"][e].cpu(), wt["W_u"][e].cpu(), wt["W_d"][e].cpu())
 
 
-def _full_check(w, x, wt, n_sample, seed):
+def _full_check(w, x, wt, n_sample, seed, n_differ=8):
     st = Stages(w, x, wt)  # the weights are already on the GPU: no copies
     st.forward()
     y_fwd = st.y.clone()
@@ -43,29 +52,35 @@ def _full_check(w, x, wt, n_sample, seed):
     assert st.device_status() == 0
     # Staged calls: same kernels and launch configurations as moe_forward.
     st.route()
+    logits = st.logits()
     st.dispatch()
-    idx = to_np(st.topk_idx)
-    check_dispatch_properties(idx, to_np(st.counts), to_np(st.offsets), to_np(st.perm_tok),
-                              to_np(st.slot_pos), w.N, w.E)
+    idx, gate = to_np(st.topk_idx), to_np(st.topk_gate)
     np.testing.assert_array_equal(to_np(st.counts), counts)
-    ffn_per_tok = (idx < w.N).sum(axis=1)
-    assert ((ffn_per_tok >= 0) & (ffn_per_tok <= w.K)).all()
     st.expert_ffn()
     st.combine()
     assert torch.equal(st.y, y_fwd)
-    # Oracle on a seeded token sample.
-    tokens = np.sort(np.random.default_rng(seed).choice(w.T, n_sample, replace=False))
-    xs = x[torch.from_numpy(tokens).to(x.device)].cpu()
+    # Whole-batch routing and dispatch against the oracle.
     W_r, b = wt["W_r"].cpu(), wt["b"].cpu()
-    ref = oracle.router(xs, W_r, b, w.K, want_scores=True)
-    near, differ = check_routing(idx[tokens], to_np(st.topk_gate)[tokens], ref, ref["scores"])
-    out = oracle.forward_sampled(np.arange(n_sample), xs, W_r, b, w.N, w.Z, w.K, _fetch(wt),
-                                 routing=ref)
-    same = (idx[tokens] == ref["topk_idx"]).all(axis=1)
+    xc = x.cpu()
+    ref = oracle.router(xc, W_r, b, w.K, want_probs=True, want_scores=True)
+    stats = check_routing_full(idx, gate, ref, logits, xc, W_r)
+    check_dispatch_vs_oracle(idx, gate, to_np(st.counts), to_np(st.offsets), to_np(st.perm_tok),
+                             to_np(st.perm_gate), to_np(st.slot_pos), w.N, w.E)
+    ffn_per_tok = (idx < w.N).sum(axis=1)
+    assert ((ffn_per_tok >= 0) & (ffn_per_tok <= w.K)).all()
+    # y: a seeded sample plus near-tie tokens the GPU routed differently, on the GPU's routing.
+    differ = np.flatnonzero((idx != ref["topk_idx"]).any(axis=1))
+    rng = np.random.default_rng(seed)
+    tokens = np.union1d(rng.choice(w.T, n_sample, replace=False),
+                        differ[rng.permutation(len(differ))[:n_differ]])
+    out = oracle.forward_sampled(np.arange(len(tokens)), oracle.bf16_bits(xc)[tokens], W_r, b,
+                                 w.N, w.Z, w.K, _fetch(wt),
+                                 routing=gpu_routing_for_oracle(idx, ref, tokens))
     y = oracle.bf16_to_f64(to_np(y_fwd))[tokens]
-    rel = assert_y_close(y[same], out["y"][same], f"{w.name} y")
-    print(f"{w.name}: mean FFN/token {ffn_per_tok.mean():.3f}, near-ties {near}/{n_sample}, "
-          f"differing {differ}, y errors {rel}")
+    rel = assert_y_close(y, out["y"], f"{w.name} y")
+    n_diff_in = int(np.isin(tokens, differ).sum())
+    print(f"{w.name}: routing {stats}; mean FFN/token {ffn_per_tok.mean():.3f}; y errors "
+          f"(max, L2) {rel} on {len(tokens)} tokens ({n_diff_in} routed differently)")
     return counts
 
 
@@ -79,6 +94,34 @@ def test_prefill_full_size(big_weights):
     w = WORKLOADS["prefill"]
     x = make_tokens(w, DEV, seed=0)
     _full_check(w, x, big_weights, n_sample=24, seed=2)
+
+
+@pytest.mark.parametrize("name", ["prefill", "skewed"])
+def test_router_logits_and_gates_whole_batch(big_weights, name):
+    """The router's fp32 logits (moe_router_logits) of every token against l = x W_r^T in fp64,
+    within the fp32 accumulation bound, and every gate against the first-order propagation of
+    those logit errors through the softmax (check_gates_against_logits).  The skewed
+    workload's Zipf term is the first term every later accumulation step rounds against, so
+    its logit and gate errors are the largest of the workloads."""
+    w = WORKLOADS[name]
+    wt = dict(big_weights)
+    if name == "skewed":
+        wt["W_r"] = apply_zipf_router(w, big_weights["W_r"].clone())
+    x = make_tokens(w, DEV, seed=0)
+    st = Stages(w, x, wt)
+    st.route()
+    logits = st.logits()
+    l_ref, mag = exact_logits(x, wt["W_r"])
+    ref = oracle.router(x.cpu(), wt["W_r"].cpu(), wt["b"].cpu(), w.K, want_probs=True,
+                        want_scores=True)
+    gate_err = check_gates_against_logits(to_np(st.topk_idx), to_np(st.topk_gate), logits, x,
+                                          wt["W_r"], ref["probs"])
+    delta = np.abs(logits - l_ref)
+    print(f"{name} router logits at d={w.d}: max|l~ - l| = {delta.max():.3e} "
+          f"= {(delta / mag).max() * 2 ** 24:.1f} u sum|xW| at most (bound "
+          f"{2 * (w.d // 16 + 16)}); max |l| {np.abs(l_ref).max():.2f}; max gate rel err "
+          f"{gate_err:.3e}")
+    assert st.device_status() == 0
 
 
 def test_skewed_pid_full_size(big_weights):
@@ -132,18 +175,17 @@ def test_decode_fp8_full_size(big_weights):
                                                 fw["s_" + k][e:e + 1].cpu().numpy())[0]
             out.append(bits)
         return tuple(out)
-    n_sample = 24
-    tokens = np.sort(np.random.default_rng(5).choice(w.T, n_sample, replace=False))
-    xs = x[torch.from_numpy(tokens).to(DEV)].cpu()
     W_r, b = big_weights["W_r"].cpu(), big_weights["b"].cpu()
-    ref = oracle.router(xs, W_r, b, w.K, want_scores=True)
-    out = oracle.forward_sampled(np.arange(n_sample), xs, W_r, b, w.N, w.Z, w.K, fetch_deq,
-                                 routing=ref)
+    ref = oracle.router(x.cpu(), W_r, b, w.K, want_probs=True, want_scores=True)
     st = Stages(w, x, big_weights)
     st.route()
-    idx = to_np(st.topk_idx)[tokens]
-    check_routing(idx, to_np(st.topk_gate)[tokens], ref, ref["scores"])
-    same = (idx == ref["topk_idx"]).all(axis=1)
+    idx = to_np(st.topk_idx)
+    check_routing_full(idx, to_np(st.topk_gate), ref, st.logits(), x, big_weights["W_r"])
+    differ = np.flatnonzero((idx != ref["topk_idx"]).any(axis=1))
+    tokens = np.union1d(np.random.default_rng(5).choice(w.T, 24, replace=False), differ[:8])
+    out = oracle.forward_sampled(np.arange(len(tokens)), oracle.bf16_bits(x.cpu())[tokens], W_r,
+                                 b, w.N, w.Z, w.K, fetch_deq,
+                                 routing=gpu_routing_for_oracle(idx, ref, tokens))
     y_s = oracle.bf16_to_f64(to_np(y))[tokens]
-    assert_y_close(y_s[same], out["y"][same], "decode fp8 y")
+    assert_y_close(y_s, out["y"], "decode fp8 y")
     del fw

@@ -89,6 +89,25 @@ def test_argument_errors_are_reported_before_any_device_work():
     assert lib.moe_last_device_error(None, None) == 1
 
 
+def test_combine_logits_and_wait_limit_argument_errors():
+    lib = mb.lib()
+    dm = mb.dims(64, 128, 8, 4, 3, 256)
+    bufs = [P(0x10000 * (i + 1)) for i in range(6)]  # x, y_perm, topk_idx, topk_gate, slot_pos, y
+    assert lib.moe_combine(ctypes.byref(dm), *bufs, None, 256, None) == 1        # no workspace
+    assert lib.moe_combine(ctypes.byref(dm), *bufs, P(0x100000), 255, None) == 4  # < status word
+    assert lib.moe_combine(ctypes.byref(dm), *bufs, P(0x100010), 256, None) == 3  # misaligned
+    assert lib.moe_combine(ctypes.byref(mb.dims(64, 100, 8, 4, 3, 256)), *bufs, P(0x100000), 256,
+                           None) == 2
+    assert lib.moe_router_logits(ctypes.byref(dm), P(0x100000), mb.scratch_size(dm), P(0),
+                                 None) == 1                                     # NULL logits
+    assert lib.moe_router_logits(ctypes.byref(dm), P(0x100000), mb.scratch_size(dm) - 1,
+                                 P(0x10000), None) == 4
+    assert lib.moe_router_logits(ctypes.byref(dm), P(0x100000), mb.scratch_size(dm),
+                                 P(0x10008), None) == 3
+    assert lib.moe_debug_set_wait_limit(-1) == 1
+    assert lib.moe_debug_set_wait_limit(0) == 0
+
+
 def test_fp8_shape_errors_before_device_work():
     lib = mb.lib()
     # R or C not a multiple of 128

@@ -62,6 +62,28 @@ def test_noalloc_dispatch_matches_workspace_dispatch_twice():
     assert mb.moe_last_device_error(ws) == 0
 
 
+def test_noalloc_dispatch_without_the_row_copy():
+    # x_perm = NULL skips the gathered copy (the fused-gather up-projection reads x itself),
+    # exactly as moe_dispatch does: the tables match and x_perm's memory is not touched.
+    T, d, N, Z, K, I = 300, 128, 8, 4, 3, 256
+    E = N + Z
+    dm = mb.dims(T, d, N, Z, K, I)
+    ws = mb.alloc_workspace(dm, DEV, scratch_only=True)
+    x = torch.randn((T, d), generator=torch.Generator().manual_seed(5)).to(torch.bfloat16).to(DEV)
+    idx, gate = _routing(T, K, E, 13)
+    want = _outputs(T, K, N, E, d)
+    got = _outputs(T, K, N, E, d)
+    got["x_perm"].fill_(3.0)
+    mb.moe_dispatch(dm, x, idx, gate, want["counts"], want["offsets"], want["perm_tok"],
+                    want["perm_gate"], want["slot_pos"], None, ws)
+    mb.moe_dispatch_noalloc(dm, x, idx, gate, got["counts"], got["offsets"], got["perm_tok"],
+                            got["perm_gate"], got["slot_pos"], None)
+    torch.cuda.synchronize()
+    for name in ("counts", "offsets", "perm_tok", "perm_gate", "slot_pos"):
+        assert torch.equal(got[name], want[name]), name
+    assert (got["x_perm"] == 3.0).all()
+
+
 def test_noalloc_dispatch_refuses_requests_beyond_its_capacity():
     # ceil(T/256) * (N+Z) must stay within 262144 counters: N+Z = 1024 allows T <= 65536.
     T, d, N, Z, K, I = 70000, 64, 512, 512, 1, 64
