@@ -292,9 +292,40 @@ __device__ __forceinline__ void signal_abort(const GemmArgs &a, volatile int *ab
 __device__ __forceinline__ float silu(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
 // ------------------------------------------------------------------ epilogue, one 32-token chunk
-// Thread `lane` of epilogue warp with TMEM lane quarter q owns output feature (q*32 + lane) of
-// each 128-row sub-tile; after the transpose through `stage` each thread stores 16 bytes of a
-// token row.
+// Stores a 32 x 32 block held one feature per lane (v[j] = feature f0 + lane of token tok0 + j)
+// as bf16 token rows.  Lanes 2i and 2i+1 trade one value per pair of tokens, so lane 2i holds
+// features (f0 + 2i, f0 + 2i + 1) of token j and lane 2i + 1 the same two features of token
+// j + 1: one packed conversion and one 4-byte shared-memory store per two values, each store
+// instruction filling two 64-byte rows of the warp's 2 KB staging area without bank conflicts;
+// then each lane copies 16 bytes of a row to global memory (four 16-byte stores per lane).
+// Every value is rounded to nearest once.
+__device__ __forceinline__ void store_rows_bf16(uint16_t *out, long long ld, int row0, int tok0,
+                                                int n_valid, int f0, int M, int lane,
+                                                const float (&v)[32], uint32_t *stage) {
+  const bool odd = (lane & 1) != 0;
+#pragma unroll
+  for (int j = 0; j < 32; j += 2) {
+    const float mine = odd ? v[j + 1] : v[j];
+    const float theirs = __shfl_xor_sync(0xffffffffu, odd ? v[j] : v[j + 1], 1);
+    stage[(j + (odd ? 1 : 0)) * 16 + (lane >> 1)] =
+        odd ? pack_bf16x2(theirs, mine) : pack_bf16x2(mine, theirs);
+  }
+  __syncwarp();
+  const int f = f0 + (lane & 3) * 8;
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int r = it * 8 + (lane >> 2);
+    const int tok = tok0 + r;
+    if (tok < n_valid && f < M) {
+      const uint4 val = *reinterpret_cast<const uint4 *>(stage + r * 16 + (lane & 3) * 4);
+      *reinterpret_cast<uint4 *>(out + (long long)(row0 + tok) * ld + f) = val;
+    }
+  }
+  __syncwarp();
+}
+
+// Thread `lane` of the epilogue warp with TMEM lane quarter q owns output feature (q*32 + lane)
+// of each 128-row sub-tile.
 template <int EPI, int BN>
 __device__ __forceinline__ void epilogue_chunk(const GemmArgs &a, const Tile &t, uint32_t tcol,
                                                int chunk, int q, int lane, float *stage) {
@@ -304,31 +335,40 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs &a, const Tile &t,
     tmem_ld_32x32b_x32(tcol, g);
     tmem_ld_32x32b_x32(tcol + BN, u);
     tmem_ld_wait();
-    uint16_t *st = reinterpret_cast<uint16_t *>(stage);
+    float h[32];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const float h = silu(__uint_as_float(g[j])) * __uint_as_float(u[j]);
-      st[j * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(h));
+    for (int j = 0; j < 32; ++j) h[j] = silu(__uint_as_float(g[j])) * __uint_as_float(u[j]);
+    store_rows_bf16(reinterpret_cast<uint16_t *>(a.out), a.out_ld, t.row0, tok0, t.n_valid,
+                    t.m0 + q * 32, a.M, lane, h, reinterpret_cast<uint32_t *>(stage));
+  } else if (EPI == kEpiGated) {
+    // The chunk's 32 gates, read by every lane as broadcast vector loads from the warp's
+    // staging area (one store per lane, eight loads) instead of 32 shuffles.
+    const int tok = tok0 + lane;
+    stage[lane] = tok >= t.n_valid ? 0.f : (a.row_scale ? __ldg(a.row_scale + t.row0 + tok) : 1.f);
+    __syncwarp();
+    float gate[32];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 g4 = reinterpret_cast<const float4 *>(stage)[i];
+      gate[4 * i] = g4.x;
+      gate[4 * i + 1] = g4.y;
+      gate[4 * i + 2] = g4.z;
+      gate[4 * i + 3] = g4.w;
     }
     __syncwarp();
-    const int f = t.m0 + q * 32 + (lane & 3) * 8;
-    uint16_t *out = reinterpret_cast<uint16_t *>(a.out);
+#pragma unroll 1
+    for (int sub = 0; sub < 2; ++sub) {
+      if (sub == 1 && !t.has_a1) break;
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tcol + sub * BN, v);
+      tmem_ld_wait();
+      float y[32];
 #pragma unroll
-    for (int it = 0; it < 4; ++it) {
-      const int r = it * 8 + (lane >> 2);
-      const int tok = tok0 + r;
-      if (tok < t.n_valid && f < a.M) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(st + r * 32 + (lane & 3) * 8);
-        *reinterpret_cast<uint4 *>(out + (long long)(t.row0 + tok) * a.out_ld + f) = v;
-      }
+      for (int j = 0; j < 32; ++j) y[j] = __uint_as_float(v[j]) * gate[j];
+      store_rows_bf16(reinterpret_cast<uint16_t *>(a.out), a.out_ld, t.row0, tok0, t.n_valid,
+                      t.m0 + sub * kBM + q * 32, a.M, lane, y, reinterpret_cast<uint32_t *>(stage));
     }
-    __syncwarp();
   } else {
-    float gate = 0.f;
-    if (EPI == kEpiGated) {
-      const int tok = tok0 + lane;
-      gate = tok >= t.n_valid ? 0.f : (a.row_scale ? __ldg(a.row_scale + t.row0 + tok) : 1.f);
-    }
 #pragma unroll 1
     for (int sub = 0; sub < 2; ++sub) {
       if (sub == 1 && !t.has_a1) break;
@@ -336,27 +376,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs &a, const Tile &t,
       tmem_ld_32x32b_x32(tcol + sub * BN, v);
       tmem_ld_wait();
       const int fbase = t.m0 + sub * kBM + q * 32;
-      if (EPI == kEpiGated) {
-        uint16_t *st = reinterpret_cast<uint16_t *>(stage);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float gj = __shfl_sync(0xffffffffu, gate, j);
-          st[j * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j]) * gj));
-        }
-        __syncwarp();
-        const int f = fbase + (lane & 3) * 8;
-        uint16_t *out = reinterpret_cast<uint16_t *>(a.out);
-#pragma unroll
-        for (int it = 0; it < 4; ++it) {
-          const int r = it * 8 + (lane >> 2);
-          const int tok = tok0 + r;
-          if (tok < t.n_valid && f < a.M) {
-            const uint4 val = *reinterpret_cast<const uint4 *>(st + r * 32 + (lane & 3) * 8);
-            *reinterpret_cast<uint4 *>(out + (long long)(t.row0 + tok) * a.out_ld + f) = val;
-          }
-        }
-        __syncwarp();
-      } else {  // kEpiF32: two passes of 16 tokens through the staging buffer
+      {  // kEpiF32: two passes of 16 tokens through the staging buffer
         const int f = fbase + (lane & 7) * 4;
         float *out = reinterpret_cast<float *>(a.out) + (long long)t.split * a.split_stride;
 #pragma unroll
@@ -463,6 +483,9 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER, PR>::kThreads, 1)
     tma_prefetch_desc(&args.map_a0);
     tma_prefetch_desc(&args.map_a1);
     tma_prefetch_desc(&args.map_a01);
+    tma_prefetch_desc(&args.map_s0);
+    tma_prefetch_desc(&args.map_s1);
+    tma_prefetch_desc(&args.map_s01);
     tma_prefetch_desc(&args.map_b256);
 #pragma unroll
     for (int i = 0; i < 4; ++i) tma_prefetch_desc(&args.map_b[i]);
@@ -509,6 +532,9 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER, PR>::kThreads, 1)
                                   : (WQ ? kQTile : kTileA) * (t.has_a1 ? 2 : 1) +
                                         (GATHER ? 0 : t.nb * kBK * 2);
         const uint64_t pol_w = t.once ? pol_w_once : pol_w_reused;
+        const CUtensorMap *map_w0 = t.once ? &args.map_s0 : &args.map_a0;
+        const CUtensorMap *map_w1 = t.once ? &args.map_s1 : &args.map_a1;
+        const CUtensorMap *map_w01 = t.once ? &args.map_s01 : &args.map_a01;
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, wlim)) {
             signal_abort(args, abort_flag);
@@ -523,10 +549,10 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER, PR>::kThreads, 1)
             const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
             if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], bytes);
             if (EPI != kEpiSwiGLU) {
-              tma_load_2d_pair(sa0, &args.map_a01, fb, kc, t.a0_row, pol_w);
+              tma_load_2d_pair(sa0, map_w01, fb, kc, t.a0_row, pol_w);
             } else {
-              tma_load_2d_pair(sa0, &args.map_a0, fb, kc, t.a0_row, pol_w);
-              tma_load_2d_pair(sa1, &args.map_a1, fb, kc, t.a1_row, pol_w);
+              tma_load_2d_pair(sa0, map_w0, fb, kc, t.a0_row, pol_w);
+              tma_load_2d_pair(sa1, map_w1, fb, kc, t.a1_row, pol_w);
             }
             const int half = t.nb >> 1, brow = t.row0 + (int)rank * half;
             int r = 0;
@@ -544,15 +570,15 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER, PR>::kThreads, 1)
           }
           mbar_arrive_expect_tx(&full_bar[stage], bytes);
           if (WQ) {  // E4M3 codes of both weight blocks at the start of the stage
-            tma_load_2d(sa0, &args.map_a0, &full_bar[stage], kc, t.a0_row, pol_w);
+            tma_load_2d(sa0, map_w0, &full_bar[stage], kc, t.a0_row, pol_w);
             if (t.has_a1)
-              tma_load_2d(sa0 + kQTile, &args.map_a1, &full_bar[stage], kc, t.a1_row, pol_w);
+              tma_load_2d(sa0 + kQTile, map_w1, &full_bar[stage], kc, t.a1_row, pol_w);
           } else if (kWideBoxes && EPI != kEpiSwiGLU && t.has_a1) {
-            tma_load_2d(sa0, &args.map_a01, &full_bar[stage], kc, t.a0_row, pol_w);
+            tma_load_2d(sa0, map_w01, &full_bar[stage], kc, t.a0_row, pol_w);
           } else {
-            tma_load_2d(sa0, &args.map_a0, &full_bar[stage], kc, t.a0_row, pol_w);
+            tma_load_2d(sa0, map_w0, &full_bar[stage], kc, t.a0_row, pol_w);
             if (t.has_a1)
-              tma_load_2d(sa1, &args.map_a1, &full_bar[stage], kc, t.a1_row, pol_w);
+              tma_load_2d(sa1, map_w1, &full_bar[stage], kc, t.a1_row, pol_w);
           }
           if (!GATHER) {
             // Token rows in boxes of 256 / 128 (as many as needed), then 64 / 32 / 16.

@@ -21,6 +21,10 @@ struct GemmArgs {
   CUtensorMap map_a1;    // W_u for SwiGLU, the same tensor as map_a0 otherwise
   CUtensorMap map_a01;   // map_a0's tensor in 64 x 256 boxes: both 128-row blocks at once when
                          // they are adjacent rows (down projection, router)
+  // The same three weight maps for tiles that read their weights exactly once (Tile::once):
+  // 256-byte L2 promotion, so each 128-byte row segment a stage requests also brings the next
+  // k-slice's segment into L2, doubling the bytes in flight of a weight-streaming tile.
+  CUtensorMap map_s0, map_s1, map_s01;
   CUtensorMap map_b[4];  // activation rows, boxes of 128 / 64 / 32 / 16 rows x 64 columns
   CUtensorMap map_b256;  // activation rows, boxes of 256 rows
   const int32_t *group_offsets;  // [num_groups + 1] activation-row offsets, or nullptr

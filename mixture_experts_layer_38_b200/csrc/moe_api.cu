@@ -123,6 +123,22 @@ bool make_act_maps(GemmArgs &a, const void *base, uint64_t rows, uint64_t cols,
   return make_map(&a.map_b256, base, rows, cols, 256, promote256);
 }
 
+// Weight maps for tiles that read their weights once: the given maps themselves when they
+// already promote to 256 bytes (or hold FP8 codes), else the same tensors with 256-byte
+// promotion (GemmArgs::map_s0).
+bool make_stream_maps(GemmArgs &a, const void *w0, const void *w1, uint64_t rows,
+                      uint64_t cols, bool promote256) {
+  if (promote256) {
+    a.map_s0 = a.map_a0;
+    a.map_s1 = a.map_a1;
+    a.map_s01 = a.map_a01;
+    return true;
+  }
+  return make_map(&a.map_s0, w0, rows, cols, 128, true) &&
+         make_map(&a.map_s1, w1, rows, cols, 128, true) &&
+         make_map(&a.map_s01, w0, rows, cols, 256, true);
+}
+
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 bool dims_ok(const moe_dims *d) {
@@ -243,7 +259,8 @@ int do_route(const moe_dims &d, const DeviceInfo &di, const Layout &L, const moe
   if (!make_map(&a.map_a0, W_r, (uint64_t)E, (uint64_t)d.d, 128, p256) ||
       !make_map(&a.map_a1, W_r, (uint64_t)E, (uint64_t)d.d, 128, p256) ||
       !make_map(&a.map_a01, W_r, (uint64_t)E, (uint64_t)d.d, 256, p256) ||
-      !make_act_maps(a, x, (uint64_t)d.T, (uint64_t)d.d, p256)) {
+      !make_act_maps(a, x, (uint64_t)d.T, (uint64_t)d.d, p256) ||
+      !make_stream_maps(a, W_r, W_r, (uint64_t)E, (uint64_t)d.d, true)) {
     return MOE_ERR_CUDA;
   }
   a.group_offsets = nullptr;
@@ -308,7 +325,9 @@ int do_expert_ffn(const moe_dims &d, const DeviceInfo &di, const Layout &L,
             make_map(&up.map_a01, W_g, (uint64_t)d.N * d.I, (uint64_t)d.d, 256, p256);
   if (!ok_w ||
       !make_act_maps(up, gather ? x : x_perm, gather ? (uint64_t)d.T : rows, (uint64_t)d.d,
-                     p256)) {
+                     p256) ||
+      !make_stream_maps(up, W_g, W_u, (uint64_t)d.N * d.I, (uint64_t)d.d,
+                        p256 || fw != nullptr)) {
     return MOE_ERR_CUDA;
   }
   up.row_index = perm_tok;
@@ -345,7 +364,9 @@ int do_expert_ffn(const moe_dims &d, const DeviceInfo &di, const Layout &L,
       : make_map(&down.map_a0, W_d, (uint64_t)d.N * d.d, (uint64_t)d.I, 128, p256) &&
             make_map(&down.map_a1, W_d, (uint64_t)d.N * d.d, (uint64_t)d.I, 128, p256) &&
             make_map(&down.map_a01, W_d, (uint64_t)d.N * d.d, (uint64_t)d.I, 256, p256);
-  if (!ok_wd || !make_act_maps(down, h, rows, (uint64_t)d.I, p256)) {
+  if (!ok_wd || !make_act_maps(down, h, rows, (uint64_t)d.I, p256) ||
+      !make_stream_maps(down, W_d, W_d, (uint64_t)d.N * d.d, (uint64_t)d.I,
+                        p256 || fw != nullptr)) {
     return MOE_ERR_CUDA;
   }
   down.group_offsets = offsets;
@@ -524,7 +545,8 @@ int moe_dense_ffn(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *W_g,
   if (!make_map(&up.map_a0, W_g, (uint64_t)d.I, (uint64_t)d.d, 128, p256) ||
       !make_map(&up.map_a1, W_u, (uint64_t)d.I, (uint64_t)d.d, 128, p256) ||
       !make_map(&up.map_a01, W_g, (uint64_t)d.I, (uint64_t)d.d, 256, p256) ||
-      !make_act_maps(up, x, (uint64_t)d.T, (uint64_t)d.d, p256)) {
+      !make_act_maps(up, x, (uint64_t)d.T, (uint64_t)d.d, p256) ||
+      !make_stream_maps(up, W_g, W_u, (uint64_t)d.I, (uint64_t)d.d, true)) {
     return MOE_ERR_CUDA;
   }
   up.group_offsets = nullptr;
@@ -542,7 +564,8 @@ int moe_dense_ffn(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *W_g,
   if (!make_map(&down.map_a0, W_d, (uint64_t)d.d, (uint64_t)d.I, 128, p256) ||
       !make_map(&down.map_a1, W_d, (uint64_t)d.d, (uint64_t)d.I, 128, p256) ||
       !make_map(&down.map_a01, W_d, (uint64_t)d.d, (uint64_t)d.I, 256, p256) ||
-      !make_act_maps(down, h, (uint64_t)d.T, (uint64_t)d.I, p256)) {
+      !make_act_maps(down, h, (uint64_t)d.T, (uint64_t)d.I, p256) ||
+      !make_stream_maps(down, W_d, W_d, (uint64_t)d.d, (uint64_t)d.I, true)) {
     return MOE_ERR_CUDA;
   }
   down.group_offsets = nullptr;
