@@ -17,7 +17,9 @@
 //
 // 256-token tiles of the FFN GEMMs run on CTA pairs (Cfg, PR): a cluster of two CTAs on two
 // SMs issues pair MMAs of M = 256 weight rows, each CTA holding half the weight rows and half
-// the token rows of a stage, so a third less shared memory feeds the same work per SM.
+// the token rows of a stage, so a third less shared memory feeds the same work per SM.  At
+// large batches the FFN GEMMs on pairs use dual_gemm_kernel (end of this file): two pipelines
+// per pair, full tiles and the lightly used experts' weight-streaming tails side by side.
 //
 // Warp roles (64 + 32 x kGemmEpiWarps = 192 threads, one CTA per SM, persistent over a static
 // tile schedule; with CTA pairs only the even CTA's warp 1 issues MMAs, whose commits signal
@@ -804,6 +806,393 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER, PR>::kThreads, 1)
   }
 }
 
+// ==================================================================== dual-pipeline CTA pairs
+// Each CTA pair runs two independent pipelines at once, each with its own shared-memory ring,
+// barriers, TMA producer, MMA issuer, four epilogue warps and TMEM columns:
+//   F  full token tiles of kDualBNF = 192 rows, and the tail of an expert when it holds more than
+//      kDualBNL rows (compute-bound: 3 stages of 2 x 16 KB weights + 96 token rows per CTA,
+//      2 x 192 accumulator columns);
+//   L  an expert's tail of at most kDualBNL = 64 rows (weight streaming: 2 stages of 2 x 16 KB
+//      weights + 32 token rows per CTA, 2 x 64 accumulator columns).
+// With one pipeline per SM every SM alternated between streaming a lightly used expert's weights
+// (tensor pipe idle) and a heavily used expert's compute-bound tiles; here both kinds of tile are
+// in flight on every SM, so HBM streaming and tensor work overlap within each SM.  Items of each
+// list are dealt round-robin over the pairs; within a token tile the weight tiles come fastest.
+constexpr int kDualBNF = 192;
+constexpr int kDualBNL = 64;
+constexpr int kDualStagesF = 3;
+constexpr int kDualStagesL = 2;
+constexpr int kDualStageF = 2 * kTileA + (kDualBNF / 2) * kBK * 2;  // 44 KB
+constexpr int kDualStageL = 2 * kTileA + (kDualBNL / 2) * kBK * 2;  // 36 KB
+constexpr int kDualEpiWarps = 4;                                     // per pipeline
+constexpr int kDualThreads = 32 * 2 * (2 + kDualEpiWarps);           // 384
+constexpr int kDualRing = kDualStagesF * kDualStageF + kDualStagesL * kDualStageL;
+constexpr int kDualStaging = 2 * kDualEpiWarps * kStagingFloats * 4;
+constexpr int kDualPrefix = 2 * (kMaxGroups + 4) * 2;               // uint16 prefixes
+constexpr int kDualBarsPerPipe = 2 * kDualStagesF + 3;
+constexpr int kDualSmemBytes = 1024 + kDualRing + kDualStaging + kDualPrefix +
+                               2 * kDualBarsPerPipe * 8 + 16;
+static_assert(kDualSmemBytes <= 232448, "shared memory per block");
+static_assert(2 * kDualBNF + 2 * kDualBNL <= kTmemCols, "TMEM holds 512 columns");
+
+struct DualSchedule {
+  const uint16_t *fpre;  // [G + 1] prefix of F tiles per group
+  const uint16_t *lpre;  // [G + 1] prefix of L tiles per group
+  int G;
+  int F, L;              // tiles of each list
+  int m_tiles;
+};
+
+__device__ __forceinline__ int find_group16(const uint16_t *pre, int G, int v) {
+  int lo = 0, hi = G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if ((int)pre[mid] <= v) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// F and L tile counts per group (rows c): F = floor(c / BNF) + (c % BNF > BNL), L = (0 < c % BNF
+// <= BNL).  The host guarantees the totals fit 16 bits (gemm_dual_fits).  Records
+// MOE_DEV_BAD_ROWS and schedules nothing if the offsets are not monotone or exceed the rows.
+__device__ void build_dual_schedule(const GemmArgs &a, uint16_t *fpre, uint16_t *lpre,
+                                    int *scratch, DualSchedule &s) {
+  const int G = a.num_groups;
+  const int per = (G + (int)blockDim.x - 1) / (int)blockDim.x;
+  const int g_begin = min(G, (int)threadIdx.x * per);
+  const int g_end = min(G, g_begin + per);
+  int nf = 0, nl = 0;
+  bool bad = false;
+  for (int g = g_begin; g < g_end; ++g) {
+    const int lo = group_off(a, g), hi = group_off(a, g + 1);
+    if (lo < 0 || hi < lo || hi > a.rows) { bad = true; continue; }
+    const int c = hi - lo, r = c % kDualBNF;
+    nf += c / kDualBNF + (r > kDualBNL ? 1 : 0);
+    nl += (r > 0 && r <= kDualBNL) ? 1 : 0;
+  }
+  int F = 0, L = 0;
+  int frun = block_exclusive_scan(nf, scratch, F);
+  int lrun = block_exclusive_scan(nl, scratch, L);
+  for (int g = g_begin; g < g_end; ++g) {
+    fpre[g] = (uint16_t)frun;
+    lpre[g] = (uint16_t)lrun;
+    const int lo = group_off(a, g), hi = group_off(a, g + 1);
+    if (!(lo < 0 || hi < lo || hi > a.rows)) {
+      const int c = hi - lo, r = c % kDualBNF;
+      frun += c / kDualBNF + (r > kDualBNL ? 1 : 0);
+      lrun += (r > 0 && r <= kDualBNL) ? 1 : 0;
+    }
+  }
+  if (threadIdx.x == 0) {
+    fpre[G] = (uint16_t)F;
+    lpre[G] = (uint16_t)L;
+  }
+  const bool any_bad = __syncthreads_or(bad);
+  if (any_bad && threadIdx.x == 0) record_status(a.status, MOE_DEV_BAD_ROWS);
+  s.fpre = fpre;
+  s.lpre = lpre;
+  s.G = G;
+  s.F = any_bad ? 0 : F;
+  s.L = any_bad ? 0 : L;
+}
+
+// Work item `item` of list F (full) or L (tail): weight tile fastest.
+template <int EPI, bool FULL>
+__device__ __forceinline__ Tile decode_dual(const GemmArgs &a, const DualSchedule &s, int item,
+                                           uint32_t rank) {
+  Tile t;
+  const int mt = item % s.m_tiles;
+  const int pos = item / s.m_tiles;
+  int g;
+  if (FULL) {
+    g = find_group16(s.fpre, s.G, pos);
+    const int lo = group_off(a, g), hi = group_off(a, g + 1);
+    t.row0 = lo + (pos - (int)s.fpre[g]) * kDualBNF;
+    t.n_valid = min(kDualBNF, hi - t.row0);
+    t.once = (hi - lo) <= kDualBNF;  // the group's only tile
+  } else {
+    g = find_group16(s.lpre, s.G, pos);
+    const int lo = group_off(a, g), hi = group_off(a, g + 1);
+    t.row0 = lo + ((hi - lo) / kDualBNF) * kDualBNF;
+    t.n_valid = hi - t.row0;
+    t.once = (hi - lo) < kDualBNF;
+  }
+  t.nb = (t.n_valid + 31) & ~31;  // a pair MMA splits N in two halves of 16k rows
+  if (EPI == kEpiSwiGLU) {
+    t.m0 = mt * 2 * kBM + (int)rank * kBM;
+    t.a0_row = g * a.M + t.m0;
+    t.a1_row = t.a0_row;
+  } else {
+    t.m0 = mt * 4 * kBM + (int)rank * 2 * kBM;
+    t.a0_row = g * a.M + t.m0;
+    t.a1_row = t.a0_row + kBM;
+  }
+  t.has_a1 = true;
+  t.kb0 = 0;
+  t.kb1 = a.K / kBK;
+  t.split = 0;
+  return t;
+}
+
+// TMA producer of one pipeline (lane 0 of its warp, both CTAs).  Each CTA loads its 128 weight
+// rows of both sub-tiles and its half of the token rows; the bytes of both CTAs complete on the
+// even CTA's stage barrier.
+template <int EPI, bool FULL, int BN, int STAGES>
+__device__ void dual_producer(const GemmArgs &args, const DualSchedule &s, uint8_t *ring,
+                              uint64_t *full_bar, uint64_t *empty_bar, volatile int *abort_flag,
+                              long long wlim, int unit, int units, uint32_t rank) {
+  constexpr int kStage = 2 * kTileA + (BN / 2) * kBK * 2;
+  const int total = (FULL ? s.F : s.L) * s.m_tiles;
+  const uint64_t pol_w_reused = l2_policy_evict_normal();
+  const uint64_t pol_w_once = l2_policy_evict_first();
+  const uint64_t pol_x = l2_policy_evict_last();
+  int stage = 0;
+  uint32_t phase = 0;
+  long long issued = 0;
+  bool ok = true;
+  for (int item = unit; ok && item < total; item += units) {
+    const Tile t = decode_dual<EPI, FULL>(args, s, item, rank);
+    const uint32_t bytes = 2u * (2 * kTileA + (t.nb / 2) * kBK * 2);
+    const uint64_t pol_w = t.once ? pol_w_once : pol_w_reused;
+    const CUtensorMap *map_w0 = t.once ? &args.map_s0 : &args.map_a0;
+    const CUtensorMap *map_w1 = t.once ? &args.map_s1 : &args.map_a1;
+    const CUtensorMap *map_w01 = t.once ? &args.map_s01 : &args.map_a01;
+    for (int kb = t.kb0; kb < t.kb1; ++kb) {
+      if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, wlim)) {
+        signal_abort(args, abort_flag);
+        ok = false;
+        break;
+      }
+      uint8_t *sa0 = ring + stage * kStage;
+      uint8_t *sa1 = sa0 + kTileA;
+      uint8_t *sb = sa0 + 2 * kTileA;
+      const int kc = kb * kBK;
+      const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
+      if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], bytes);
+      if (EPI != kEpiSwiGLU) {
+        tma_load_2d_pair(sa0, map_w01, fb, kc, t.a0_row, pol_w);
+      } else {
+        tma_load_2d_pair(sa0, map_w0, fb, kc, t.a0_row, pol_w);
+        tma_load_2d_pair(sa1, map_w1, fb, kc, t.a1_row, pol_w);
+      }
+      const int half = t.nb >> 1, brow = t.row0 + (int)rank * half;
+      int r = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int box = 128 >> i;
+        if (half - r >= box) {
+          tma_load_2d_pair(sb + r * (kBK * 2), &args.map_b[i], fb, kc, brow + r, pol_x);
+          r += box;
+        }
+      }
+      ++issued;
+      if (++stage == STAGES) { stage = 0; phase ^= 1; }
+    }
+  }
+  if (!ok && rank == 0) {
+    // Drain the copies that may still be landing in the ring (bounded; the even CTA's
+    // barriers count both CTAs' copies).
+    for (long long i = 1; i <= issued && i <= STAGES; ++i) {
+      const long long idx = issued - i;
+      const int st = (int)(idx % STAGES);
+      const uint32_t par = (uint32_t)((idx / STAGES) & 1);
+      const long long t0 = clock64();
+      while (!mbar_try_wait(&full_bar[st], par) && clock64() - t0 < kDrainLimitCycles) {}
+    }
+  }
+}
+
+// MMA issuer of one pipeline (lane 0 of its warp, even CTA): pair MMAs (M = 256 weight rows,
+// N = the tile's rows rounded to 32) into the pipeline's two accumulators at TMEM column `col`.
+template <int EPI, bool FULL, int BN, int STAGES>
+__device__ void dual_mma(const GemmArgs &args, const DualSchedule &s, uint8_t *ring,
+                         uint64_t *full_bar, uint64_t *empty_bar, uint64_t *tfull_bar,
+                         uint64_t *tempty_bar, uint64_t *drain_bar, volatile int *abort_flag,
+                         long long wlim, int unit, int units, uint32_t tmem_base, int col) {
+  constexpr int kStage = 2 * kTileA + (BN / 2) * kBK * 2;
+  const int total = (FULL ? s.F : s.L) * s.m_tiles;
+  int stage = 0;
+  uint32_t phase = 0;
+  int it = 0;
+  bool ok = true;
+  bool any = false;
+  for (int item = unit; ok && item < total; item += units, ++it) {
+    const Tile t = decode_dual<EPI, FULL>(args, s, item, 0);
+    if (!mbar_wait(tempty_bar, (it & 1) ^ 1, abort_flag, wlim)) {
+      signal_abort(args, abort_flag);
+      ok = false;
+      break;
+    }
+    tc_fence_after();
+    const uint32_t d0 = tmem_base + col;
+    const uint32_t d1 = d0 + BN;
+    const uint32_t idesc = idesc_bf16_f32(2 * kBM, t.nb);
+    for (int kb = t.kb0; kb < t.kb1; ++kb) {
+      if (!mbar_wait(&full_bar[stage], phase, abort_flag, wlim)) {
+        signal_abort(args, abort_flag);
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t abase = smem_u32(ring + stage * kStage);
+      const uint32_t bbase = abase + 2 * kTileA;
+#pragma unroll
+      for (int k = 0; k < kBK / 16; ++k) {
+        const uint64_t bdesc = sw128_kmajor_desc(bbase + k * 32);
+        const uint32_t acc = (kb > t.kb0 || k > 0) ? 1u : 0u;
+        umma_bf16_pair(d0, sw128_kmajor_desc(abase + k * 32), bdesc, idesc, acc);
+        umma_bf16_pair(d1, sw128_kmajor_desc(abase + kTileA + k * 32), bdesc, idesc, acc);
+      }
+      any = true;
+      umma_commit_pair(&empty_bar[stage], 0x3);  // frees the stage in both CTAs
+      if (++stage == STAGES) { stage = 0; phase ^= 1; }
+    }
+    if (!ok) break;
+    umma_commit_pair(tfull_bar, 0x3);
+  }
+  if (!ok && any) {
+    umma_commit_pair(drain_bar, 0x1);
+    const long long t0 = clock64();
+    while (!mbar_try_wait(drain_bar, 0) && clock64() - t0 < kDrainLimitCycles) {}
+  }
+}
+
+// Epilogue warp of one pipeline (both CTAs): drains its lane quarter of the accumulators at TMEM
+// column `col` and releases them on the even CTA's barrier.
+template <int EPI, bool FULL, int BN>
+__device__ void dual_epilogue(const GemmArgs &args, const DualSchedule &s, uint64_t *tfull_bar,
+                              uint64_t *tempty_bar, volatile int *abort_flag, long long wlim,
+                              int unit, int units, uint32_t rank, uint32_t tmem_base, int col,
+                              int q, int lane, float *stage) {
+  const int total = (FULL ? s.F : s.L) * s.m_tiles;
+  int it = 0;
+  for (int item = unit; item < total; item += units, ++it) {
+    const Tile t = decode_dual<EPI, FULL>(args, s, item, rank);
+    if (!warp_wait(tfull_bar, it & 1, abort_flag, wlim)) {
+      if (lane == 0) signal_abort(args, abort_flag);
+      break;
+    }
+    tc_fence_after();
+    const uint32_t tcol = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + col;
+    const int chunks = (t.n_valid + 31) / 32;
+    for (int c = 0; c < chunks; ++c)
+      epilogue_chunk<EPI, BN>(args, t, tcol + c * 32, c, q, lane, stage);
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(tempty_bar), 0));
+  }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kDualThreads, 1)
+    dual_gemm_kernel(const __grid_constant__ GemmArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *ring_f = smem;
+  uint8_t *ring_l = smem + kDualStagesF * kDualStageF;
+  float *staging = reinterpret_cast<float *>(smem + kDualRing);
+  uint16_t *fpre = reinterpret_cast<uint16_t *>(smem + kDualRing + kDualStaging);
+  uint16_t *lpre = fpre + kMaxGroups + 4;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kDualRing + kDualStaging + kDualPrefix);
+  // per pipeline p: full[kDualStagesF], empty[kDualStagesF], tfull, tempty, drain
+  uint64_t *bf = bars, *bl = bars + kDualBarsPerPipe;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * kDualBarsPerPipe);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int unit = (int)(blockIdx.x >> 1);
+  const int units = (int)(gridDim.x >> 1);
+
+  if (threadIdx.x == 0) {
+    for (int p = 0; p < 2; ++p) {
+      uint64_t *b = p ? bl : bf;
+      const int stages = p ? kDualStagesL : kDualStagesF;
+      for (int i = 0; i < stages; ++i) {
+        mbar_init(&b[i], 1);
+        mbar_init(&b[kDualStagesF + i], 1);
+      }
+      mbar_init(&b[2 * kDualStagesF], 1);                       // tfull
+      mbar_init(&b[2 * kDualStagesF + 1], 2 * kDualEpiWarps);   // tempty: both CTAs' epilogues
+      mbar_init(&b[2 * kDualStagesF + 2], 1);                   // drain
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&args.map_a0);
+    tma_prefetch_desc(&args.map_a1);
+    tma_prefetch_desc(&args.map_a01);
+    tma_prefetch_desc(&args.map_s0);
+    tma_prefetch_desc(&args.map_s1);
+    tma_prefetch_desc(&args.map_s01);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) tma_prefetch_desc(&args.map_b[i]);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  DualSchedule sched;
+  build_dual_schedule(args, fpre, lpre, reinterpret_cast<int *>(staging), sched);
+  sched.m_tiles = m_tiles_of<EPI, true>(args.M);
+  const long long wlim = args.wait_limit > 0 ? args.wait_limit : kWaitLimitCycles;
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers initialised before any remote arrival
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  constexpr int kColF = 0, kColL = 2 * kDualBNF;
+
+  const int role = warp % 6;           // 0 producer, 1 MMA, 2-5 epilogue
+  const bool full = warp < 6;
+  uint64_t *b = full ? bf : bl;
+  if (role == 0) {
+    if (lane == 0) {
+      if (full)
+        dual_producer<EPI, true, kDualBNF, kDualStagesF>(args, sched, ring_f, b, b + kDualStagesF,
+                                                         abort_flag, wlim, unit, units, rank);
+      else
+        dual_producer<EPI, false, kDualBNL, kDualStagesL>(args, sched, ring_l, b,
+                                                          b + kDualStagesF, abort_flag, wlim,
+                                                          unit, units, rank);
+    }
+  } else if (role == 1) {
+    if (lane == 0 && rank == 0) {
+      if (full)
+        dual_mma<EPI, true, kDualBNF, kDualStagesF>(
+            args, sched, ring_f, b, b + kDualStagesF, b + 2 * kDualStagesF,
+            b + 2 * kDualStagesF + 1, b + 2 * kDualStagesF + 2, abort_flag, wlim, unit, units,
+            tmem_base, kColF);
+      else
+        dual_mma<EPI, false, kDualBNL, kDualStagesL>(
+            args, sched, ring_l, b, b + kDualStagesF, b + 2 * kDualStagesF,
+            b + 2 * kDualStagesF + 1, b + 2 * kDualStagesF + 2, abort_flag, wlim, unit, units,
+            tmem_base, kColL);
+    }
+  } else {
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    float *stage = staging + (warp - (full ? 2 : 4)) * kStagingFloats;
+    if (full)
+      dual_epilogue<EPI, true, kDualBNF>(args, sched, b + 2 * kDualStagesF,
+                                         b + 2 * kDualStagesF + 1, abort_flag, wlim, unit, units,
+                                         rank, tmem_base, kColF, q, lane, stage);
+    else
+      dual_epilogue<EPI, false, kDualBNL>(args, sched, b + 2 * kDualStagesF,
+                                          b + 2 * kDualStagesF + 1, abort_flag, wlim, unit,
+                                          units, rank, tmem_base, kColL, q, lane, stage);
+  }
+
+  tc_fence_before();
+  __syncwarp();    // lanes 1-31 of the producer and MMA warps skipped the role loops: reconverge
+  cluster_sync();  // no CTA leaves while its peer may still touch its barriers or memory
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
 template <int EPI, int BN, bool WQ = false, bool GATHER = false, bool PR = false>
 cudaError_t set_smem_limit() {
   return cudaFuncSetAttribute(grouped_gemm_kernel<EPI, BN, WQ, GATHER, PR>,
@@ -855,6 +1244,32 @@ cudaError_t prepare_pair(int device) {
   return cudaSuccess;
 }
 
+int g_max_dual_pairs[kMaxDevices] = {0};
+
+cudaLaunchConfig_t dual_config(int pairs, cudaStream_t stream, cudaLaunchAttribute *attr) {
+  cudaLaunchConfig_t cfg = pair_config(pairs, stream, attr);
+  cfg.blockDim = dim3(kDualThreads, 1, 1);
+  cfg.dynamicSmemBytes = kDualSmemBytes;
+  return cfg;
+}
+
+template <int EPI>
+cudaError_t prepare_dual(int device) {
+  cudaError_t e = cudaFuncSetAttribute(dual_gemm_kernel<EPI>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kDualSmemBytes);
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[1];
+  const cudaLaunchConfig_t cfg = dual_config(1, nullptr, attr);
+  int clusters = 0;
+  e = cudaOccupancyMaxActiveClusters(&clusters, dual_gemm_kernel<EPI>, &cfg);
+  if (e != cudaSuccess) return e;
+  if (clusters <= 0) return cudaErrorInvalidConfiguration;
+  if (g_max_dual_pairs[device] == 0 || clusters < g_max_dual_pairs[device])
+    g_max_dual_pairs[device] = clusters;
+  return cudaSuccess;
+}
+
 template <int BN>
 cudaError_t launch_bn(int epi, const GemmArgs &args_in, int grid, cudaStream_t stream) {
   const GemmArgs args = with_limit(args_in);
@@ -883,6 +1298,8 @@ cudaError_t launch_bn(int epi, const GemmArgs &args_in, int grid, cudaStream_t s
 cudaError_t gemm_prepare(int device) {
   if (device < 0 || device >= kMaxDevices) return cudaErrorInvalidDevice;
   cudaError_t e;
+  if ((e = prepare_dual<kEpiSwiGLU>(device)) != cudaSuccess) return e;
+  if ((e = prepare_dual<kEpiGated>(device)) != cudaSuccess) return e;
   if ((e = prepare_pair<kEpiSwiGLU>(device)) != cudaSuccess) return e;
   if ((e = prepare_pair<kEpiGated>(device)) != cudaSuccess) return e;
   if ((e = set_smem_limit<kEpiSwiGLU, 128>()) != cudaSuccess) return e;
@@ -910,6 +1327,28 @@ int gemm_tile_tokens(long long rows, int groups, int K) {
 
 int gemm_max_pairs(int device) {
   return (device >= 0 && device < kMaxDevices) ? g_max_pairs[device] : 0;
+}
+
+int gemm_max_dual_pairs(int device) {
+  return (device >= 0 && device < kMaxDevices) ? g_max_dual_pairs[device] : 0;
+}
+
+bool gemm_dual_fits(long long rows, int groups) {
+  // Per-group tile prefixes are 16-bit: F tiles <= rows / 192 + groups, L tiles <= groups.
+  return groups <= kMaxGroups && rows / kDualBNF + groups + 8 < 65536;
+}
+
+cudaError_t launch_grouped_gemm_dual(int epi, const GemmArgs &args_in, int pairs,
+                                     cudaStream_t stream) {
+  if (pairs <= 0) return cudaErrorInvalidConfiguration;
+  const GemmArgs args = with_limit(args_in);
+  cudaLaunchAttribute attr[1];
+  const cudaLaunchConfig_t cfg = dual_config(pairs, stream, attr);
+  switch (epi) {
+    case kEpiSwiGLU: return cudaLaunchKernelEx(&cfg, dual_gemm_kernel<kEpiSwiGLU>, args);
+    case kEpiGated: return cudaLaunchKernelEx(&cfg, dual_gemm_kernel<kEpiGated>, args);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t launch_grouped_gemm_pair(int epi, const GemmArgs &args_in, int pairs,

@@ -114,13 +114,21 @@ def test_expert_ffn_matches_oracle(name):
     assert st.device_status() == 0
 
 
-@pytest.mark.parametrize("I", [512, 384])
-def test_expert_ffn_wide_tiles_matches_oracle(I):
-    # d = 4096 with >= 128 rows per expert selects 256-token tiles: I = 512 runs them on CTA
-    # pairs (I a multiple of 256, d of 512), I = 384 on single CTAs.  Ragged groups built
-    # directly: full 256-row tiles with and without tails, tail-only experts (100 / 30 / 17 /
-    # 1 rows), an empty expert; 1224 rows = 306 tokens x K = 4.
-    counts = np.array([520, 300, 256, 100, 17, 1, 0, 30])
+@pytest.mark.parametrize("I,counts", [
+    (512, (520, 300, 256, 100, 17, 1, 0, 30)),
+    (384, (520, 300, 256, 100, 17, 1, 0, 30)),
+    (512, (192, 193, 65, 64, 384, 257, 0, 129)),
+])
+def test_expert_ffn_wide_tiles_matches_oracle(I, counts):
+    # d = 4096 with >= 128 rows per expert selects the wide tiles: I = 512 runs them on CTA
+    # pairs (I a multiple of 256, d of 512) with the two-pipeline kernel (192-row full tiles
+    # and tails over 64 rows in one pipeline, tails of at most 64 rows in the other), I = 384
+    # on single CTAs with 256-token tiles.  Ragged groups built directly: several full tiles
+    # with and without tails, tail-only experts (100 / 30 / 17 / 1 rows), an empty expert; the
+    # third case sits on the two-pipeline kernel's boundaries (192 = one full tile, 193 = one
+    # full tile + a 1-row tail, 65 = the smallest tail kept in the full-tile pipeline, 64 = the
+    # largest in the tail pipeline, 384, 257 = 192 + 65, 129).  Rows = K = 4 times the tokens.
+    counts = np.array(counts)
     R = int(counts.sum())
     w = Workload("wide", T=R // 4, d=4096, N=8, Z=4, K=4, I=I)
     wt = make_weights(w, seed=5)
