@@ -15,11 +15,10 @@
 // the gate and the up value of one feature and SwiGLU needs no data exchange.  For the down
 // projection and the router they are 256 consecutive output rows.
 //
-// 256-token tiles of the FFN GEMMs run on CTA pairs (Cfg, PR): a cluster of two CTAs on two
-// SMs issues pair MMAs of M = 256 weight rows, each CTA holding half the weight rows and half
-// the token rows of a stage, so a third less shared memory feeds the same work per SM.  At
-// large batches the FFN GEMMs on pairs use dual_gemm_kernel (end of this file): two pipelines
-// per pair, full tiles and the lightly used experts' weight-streaming tails side by side.
+// At large batches the FFN GEMMs run on CTA pairs instead (dual_gemm_kernel, second half of this
+// file): a cluster of two CTAs on two SMs issues pair MMAs of M = 256 weight rows, each CTA
+// holding half the weight rows and half the token rows of a stage, and each pair runs two
+// pipelines at once, full tiles beside the lightly used experts' weight-streaming tails.
 //
 // Warp roles (64 + 32 x kGemmEpiWarps = 192 threads, one CTA per SM, persistent over a static
 // tile schedule; with CTA pairs only the even CTA's warp 1 issues MMAs, whose commits signal
@@ -87,17 +86,10 @@ constexpr int kConvWarps = 8;
 constexpr int kLoadWarps = 4;
 constexpr int kLoadThreads = 32 * kLoadWarps;
 
-// CTA pairs (PR, used with BN = 256): a cluster of two CTAs on two SMs computes a tile of
-// 2 x 256 weight rows x up to 256 tokens with pair MMAs (M = 256).  CTA r holds weight rows
-// [128 r, 128 r + 128) of each 256-row sub-tile and token rows [r nb/2, (r+1) nb/2) of the tile
-// in its own 48 KB stages (4 in the ring); the even CTA issues the MMAs, which read both CTAs'
-// operands and leave each CTA's 128 rows x nb columns in its own TMEM.  Per SM and k-step,
-// 48 KB of shared memory feed the work that takes 64 KB in a single-CTA 256-token tile.
-template <int BN, bool WQ = false, bool GA = false, bool PR = false>
+template <int BN, bool WQ = false, bool GA = false>
 struct Cfg {
-  static_assert(!PR || (BN == 256 && !WQ && !GA), "CTA pairs: 256-token tiled loads only");
   static constexpr int kAccBufs = BN <= 128 ? 2 : 1;
-  static constexpr int kStage = (WQ ? 2 * kQTile : 2 * kTileA) + (PR ? BN / 2 : BN) * kBK * 2;
+  static constexpr int kStage = (WQ ? 2 * kQTile : 2 * kTileA) + BN * kBK * 2;
   static constexpr int kCSlots = WQ ? 2 : 0;              // bf16 weight slots
   static constexpr int kCRing = kCSlots * 2 * kTileA;
   static constexpr int kStages = (192 * 1024 - kCRing) / kStage;
@@ -158,9 +150,8 @@ __device__ __forceinline__ int find_group(const int *pre, int G, int v) {
   return lo;
 }
 
-template <int EPI, int BN, bool PR = false>
-__device__ __forceinline__ Tile decode_tile(const GemmArgs &a, const Schedule &s, int tile,
-                                            uint32_t rank = 0) {
+template <int EPI, int BN>
+__device__ __forceinline__ Tile decode_tile(const GemmArgs &a, const Schedule &s, int tile) {
   Tile t;
   const int mt = tile % s.m_tiles;
   const int rest = tile / s.m_tiles;
@@ -183,18 +174,17 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs &a, const Schedule &s
     t.n_valid = BN;
     t.once = false;
   }
-  // A pair MMA splits N in two halves of a multiple of 16 rows each.
-  t.nb = PR ? (t.n_valid + 31) & ~31 : (t.n_valid + 15) & ~15;
+  t.nb = (t.n_valid + 15) & ~15;
   if (EPI == kEpiSwiGLU) {
-    t.m0 = PR ? mt * 2 * kBM + (int)rank * kBM : mt * kBM;
+    t.m0 = mt * kBM;
     t.a0_row = g * a.M + t.m0;
     t.a1_row = t.a0_row;
     t.has_a1 = true;
   } else {
-    t.m0 = PR ? mt * 4 * kBM + (int)rank * 2 * kBM : mt * 2 * kBM;
+    t.m0 = mt * 2 * kBM;
     t.a0_row = g * a.M + t.m0;
     t.a1_row = t.a0_row + kBM;
-    t.has_a1 = PR || (t.m0 + kBM) < a.M;  // a pair always fills both (M divides evenly)
+    t.has_a1 = (t.m0 + kBM) < a.M;
   }
   const int kblocks = a.K / kBK;
   t.kb0 = (int)(((long long)kblocks * t.split) / s.splits);
@@ -268,9 +258,9 @@ __device__ bool build_schedule(const GemmArgs &a, int *hpre, int *lpre, int *scr
   return !any_bad;
 }
 
-template <int EPI, bool PR = false>
+template <int EPI>
 __device__ __forceinline__ int m_tiles_of(int M) {
-  const int rows = (EPI == kEpiSwiGLU ? kBM : 2 * kBM) * (PR ? 2 : 1);
+  const int rows = EPI == kEpiSwiGLU ? kBM : 2 * kBM;
   return (M + rows - 1) / rows;
 }
 
@@ -433,10 +423,10 @@ __device__ __forceinline__ void convert_fp8_block(const uint8_t *q, uint8_t *dst
   }
 }
 
-template <int EPI, int BN, bool WQ, bool GATHER, bool PR = false>
-__global__ void __launch_bounds__(Cfg<BN, WQ, GATHER, PR>::kThreads, 1)
+template <int EPI, int BN, bool WQ, bool GATHER>
+__global__ void __launch_bounds__(Cfg<BN, WQ, GATHER>::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ GemmArgs args) {
-  using C = Cfg<BN, WQ, GATHER, PR>;
+  using C = Cfg<BN, WQ, GATHER>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -459,10 +449,8 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER, PR>::kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // Tiles are dealt to CTAs, or with CTA pairs to pairs (both CTAs walk the same tiles).
-  const uint32_t rank = PR ? cluster_ctarank() : 0u;
-  const int unit = PR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
-  const int units = PR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  const int unit = (int)blockIdx.x;
+  const int units = (int)gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -471,7 +459,7 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER, PR>::kThreads, 1)
     }
     for (int b = 0; b < C::kAccBufs; ++b) {
       mbar_init(&tfull_bar[b], 1);
-      mbar_init(&tempty_bar[b], (PR ? 2 : 1) * kEpiWarps);  // PR: both CTAs' epilogues
+      mbar_init(&tempty_bar[b], kEpiWarps);
     }
     mbar_init(drain_bar, 1);
     for (int c = 0; c < C::kCSlots; ++c) {
@@ -493,23 +481,17 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER, PR>::kThreads, 1)
     for (int i = 0; i < 4; ++i) tma_prefetch_desc(&args.map_b[i]);
   }
   if (warp == 1) {
-    if (PR) {
-      tmem_alloc_pair(tmem_slot, kTmemCols);
-      tmem_relinquish_pair();
-    } else {
-      tmem_alloc(tmem_slot, kTmemCols);
-      tmem_relinquish();
-    }
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
   }
   Schedule sched;
   build_schedule<BN>(args, hpre, lpre, reinterpret_cast<int *>(staging), sched);
-  sched.m_tiles = m_tiles_of<EPI, PR>(args.M);
+  sched.m_tiles = m_tiles_of<EPI>(args.M);
   sched.splits = EPI == kEpiF32 ? args.k_splits : 1;
   sched.total = sched.total * sched.m_tiles * sched.splits;
   const long long wlim = args.wait_limit > 0 ? args.wait_limit : kWaitLimitCycles;
   tc_fence_before();
-  if (PR) cluster_sync();  // both CTAs' barriers initialised before any remote arrival
-  else __syncthreads();
+  __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -528,11 +510,9 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER, PR>::kThreads, 1)
       long long issued = 0;
       bool ok = true;
       for (int tile = unit; ok && tile < sched.total; tile += units) {
-        const Tile t = decode_tile<EPI, BN, PR>(args, sched, tile, rank);
-        // PR: the even CTA's stage barrier counts both CTAs' bytes (equal halves).
-        const uint32_t bytes = PR ? 2u * (2 * kTileA + (t.nb / 2) * kBK * 2)
-                                  : (WQ ? kQTile : kTileA) * (t.has_a1 ? 2 : 1) +
-                                        (GATHER ? 0 : t.nb * kBK * 2);
+        const Tile t = decode_tile<EPI, BN>(args, sched, tile);
+        const uint32_t bytes = (WQ ? kQTile : kTileA) * (t.has_a1 ? 2 : 1) +
+                               (GATHER ? 0 : t.nb * kBK * 2);
         const uint64_t pol_w = t.once ? pol_w_once : pol_w_reused;
         const CUtensorMap *map_w0 = t.once ? &args.map_s0 : &args.map_a0;
         const CUtensorMap *map_w1 = t.once ? &args.map_s1 : &args.map_a1;
@@ -547,29 +527,6 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER, PR>::kThreads, 1)
           uint8_t *sa1 = sa0 + kTileA;
           uint8_t *sb = sa0 + (WQ ? 2 * kQTile : 2 * kTileA);
           const int kc = kb * kBK;
-          if (PR) {
-            const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
-            if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], bytes);
-            if (EPI != kEpiSwiGLU) {
-              tma_load_2d_pair(sa0, map_w01, fb, kc, t.a0_row, pol_w);
-            } else {
-              tma_load_2d_pair(sa0, map_w0, fb, kc, t.a0_row, pol_w);
-              tma_load_2d_pair(sa1, map_w1, fb, kc, t.a1_row, pol_w);
-            }
-            const int half = t.nb >> 1, brow = t.row0 + (int)rank * half;
-            int r = 0;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int box = 128 >> i;
-              if (half - r >= box) {
-                tma_load_2d_pair(sb + r * (kBK * 2), &args.map_b[i], fb, kc, brow + r, pol_x);
-                r += box;
-              }
-            }
-            ++issued;
-            if (++stage == C::kStages) { stage = 0; phase ^= 1; }
-            continue;
-          }
           mbar_arrive_expect_tx(&full_bar[stage], bytes);
           if (WQ) {  // E4M3 codes of both weight blocks at the start of the stage
             tma_load_2d(sa0, map_w0, &full_bar[stage], kc, t.a0_row, pol_w);
@@ -606,9 +563,8 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER, PR>::kThreads, 1)
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
         }
       }
-      if (!ok && !(PR && rank != 0)) {
-        // Drain the copies that may still be landing in the ring (bounded; with CTA pairs the
-        // even CTA's barriers count both CTAs' copies).
+      if (!ok) {
+        // Drain the copies that may still be landing in the ring (bounded).
         for (long long i = 1; i <= issued && i <= C::kStages; ++i) {
           const long long idx = issued - i;
           const int s = (int)(idx % C::kStages);
@@ -620,7 +576,7 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER, PR>::kThreads, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0 && rank == 0) {
+    if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       int cslot = 0;            // WQ: bf16 slot of the current k-step
@@ -629,7 +585,7 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER, PR>::kThreads, 1)
       bool ok = true;
       bool any = false;
       for (int tile = unit; ok && tile < sched.total; tile += units, ++it) {
-        const Tile t = decode_tile<EPI, BN, PR>(args, sched, tile, rank);
+        const Tile t = decode_tile<EPI, BN>(args, sched, tile);
         const int buf = it % C::kAccBufs;
         const uint32_t use = (uint32_t)(it / C::kAccBufs);
         if (!mbar_wait(&tempty_bar[buf], (use & 1) ^ 1, abort_flag, wlim)) {
@@ -640,7 +596,7 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER, PR>::kThreads, 1)
         tc_fence_after();
         const uint32_t d0 = tmem_base + buf * (2 * BN);
         const uint32_t d1 = d0 + BN;
-        const uint32_t idesc = idesc_bf16_f32(PR ? 2 * kBM : kBM, t.nb);
+        const uint32_t idesc = idesc_bf16_f32(kBM, t.nb);
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
           if (!mbar_wait(&full_bar[stage], phase, abort_flag, wlim) ||
               (WQ && !mbar_wait(&cfull_bar[cslot], cphase, abort_flag, wlim))) {
@@ -659,18 +615,12 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER, PR>::kThreads, 1)
           for (int k = 0; k < kBK / 16; ++k) {
             const uint64_t bdesc = sw128_kmajor_desc(bbase + k * 32);
             const uint32_t acc = (kb > t.kb0 || k > 0) ? 1u : 0u;
-            if (PR) {
-              umma_bf16_pair(d0, sw128_kmajor_desc(abase + k * 32), bdesc, idesc, acc);
-              umma_bf16_pair(d1, sw128_kmajor_desc(abase + kTileA + k * 32), bdesc, idesc, acc);
-            } else {
-              umma_bf16(d0, sw128_kmajor_desc(abase + k * 32), bdesc, idesc, acc);
-              if (t.has_a1)
-                umma_bf16(d1, sw128_kmajor_desc(abase + kTileA + k * 32), bdesc, idesc, acc);
-            }
+            umma_bf16(d0, sw128_kmajor_desc(abase + k * 32), bdesc, idesc, acc);
+            if (t.has_a1)
+              umma_bf16(d1, sw128_kmajor_desc(abase + kTileA + k * 32), bdesc, idesc, acc);
           }
           any = true;
-          if (PR) umma_commit_pair(&empty_bar[stage], 0x3);  // frees the stage in both CTAs
-          else umma_commit(&empty_bar[stage]);
+          umma_commit(&empty_bar[stage]);
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
           if (WQ) {
             umma_commit(&cempty_bar[cslot]);
@@ -678,12 +628,10 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER, PR>::kThreads, 1)
           }
         }
         if (!ok) break;
-        if (PR) umma_commit_pair(&tfull_bar[buf], 0x3);
-        else umma_commit(&tfull_bar[buf]);
+        umma_commit(&tfull_bar[buf]);
       }
       if (!ok && any) {
-        if (PR) umma_commit_pair(drain_bar, 0x1);
-        else umma_commit(drain_bar);
+        umma_commit(drain_bar);
         const long long t0 = clock64();
         while (!mbar_try_wait(drain_bar, 0) && clock64() - t0 < kDrainLimitCycles) {}
       }
@@ -771,7 +719,7 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER, PR>::kThreads, 1)
     float *stage = staging + (warp - 2) * kStagingFloats;
     int it = 0;
     for (int tile = unit; tile < sched.total; tile += units, ++it) {
-      const Tile t = decode_tile<EPI, BN, PR>(args, sched, tile, rank);
+      const Tile t = decode_tile<EPI, BN>(args, sched, tile);
       const int buf = it % C::kAccBufs;
       const uint32_t use = (uint32_t)(it / C::kAccBufs);
       if (!warp_wait(&tfull_bar[buf], use & 1, abort_flag, wlim)) {
@@ -785,24 +733,15 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER, PR>::kThreads, 1)
         epilogue_chunk<EPI, BN>(args, t, tcol + c * 32, c, q, lane, stage);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        if (PR) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty_bar[buf]), 0));
-        else mbar_arrive(&tempty_bar[buf]);
-      }
+      if (lane == 0) mbar_arrive(&tempty_bar[buf]);
     }
   }
 
   tc_fence_before();
-  if (PR) {
-    __syncwarp();    // lanes 1-31 of warps 0 and 1 skipped the role loops: reconverge
-    cluster_sync();  // no CTA leaves while its peer may still touch its barriers or memory
-  } else {
-    __syncthreads();
-  }
+  __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    if (PR) tmem_dealloc_pair(tmem_base, kTmemCols);
-    else tmem_dealloc(tmem_base, kTmemCols);
+    tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 
@@ -1137,7 +1076,9 @@ __global__ void __launch_bounds__(kDualThreads, 1)
   }
   DualSchedule sched;
   build_dual_schedule(args, fpre, lpre, reinterpret_cast<int *>(staging), sched);
-  sched.m_tiles = m_tiles_of<EPI, true>(args.M);
+  // Weight rows per pair tile: 2 x 128 features (gate and up rows of each) for the
+  // up-projection, 2 x 2 x 128 output rows for the down-projection.
+  sched.m_tiles = (args.M + (EPI == kEpiSwiGLU ? 2 : 4) * kBM - 1) / ((EPI == kEpiSwiGLU ? 2 : 4) * kBM);
   const long long wlim = args.wait_limit > 0 ? args.wait_limit : kWaitLimitCycles;
   tc_fence_before();
   cluster_sync();  // both CTAs' barriers initialised before any remote arrival
@@ -1193,11 +1134,11 @@ __global__ void __launch_bounds__(kDualThreads, 1)
   }
 }
 
-template <int EPI, int BN, bool WQ = false, bool GATHER = false, bool PR = false>
+template <int EPI, int BN, bool WQ = false, bool GATHER = false>
 cudaError_t set_smem_limit() {
-  return cudaFuncSetAttribute(grouped_gemm_kernel<EPI, BN, WQ, GATHER, PR>,
+  return cudaFuncSetAttribute(grouped_gemm_kernel<EPI, BN, WQ, GATHER>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              Cfg<BN, WQ, GATHER, PR>::kSmemBytes);
+                              Cfg<BN, WQ, GATHER>::kSmemBytes);
 }
 
 // Wait limit applied to launches (0: kWaitLimitCycles); only the timeout-path tests change it.
@@ -1209,15 +1150,15 @@ GemmArgs with_limit(const GemmArgs &args) {
   return a;
 }
 
-using PairCfg = Cfg<256, false, false, true>;
 constexpr int kMaxDevices = 64;
-int g_max_pairs[kMaxDevices] = {0};
+int g_max_dual_pairs[kMaxDevices] = {0};
 
-cudaLaunchConfig_t pair_config(int pairs, cudaStream_t stream, cudaLaunchAttribute *attr) {
+// Clusters of two CTAs (one CTA pair per cluster) of the two-pipeline kernel.
+cudaLaunchConfig_t dual_config(int pairs, cudaStream_t stream, cudaLaunchAttribute *attr) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cfg.blockDim = dim3(PairCfg::kThreads, 1, 1);
-  cfg.dynamicSmemBytes = PairCfg::kSmemBytes;
+  cfg.blockDim = dim3(kDualThreads, 1, 1);
+  cfg.dynamicSmemBytes = kDualSmemBytes;
   cfg.stream = stream;
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
@@ -1225,31 +1166,6 @@ cudaLaunchConfig_t pair_config(int pairs, cudaStream_t stream, cudaLaunchAttribu
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cfg;
-}
-
-// Shared-memory limit of a pair instantiation, and the pairs that can be resident at once.
-template <int EPI>
-cudaError_t prepare_pair(int device) {
-  cudaError_t e = set_smem_limit<EPI, 256, false, false, true>();
-  if (e != cudaSuccess) return e;
-  cudaLaunchAttribute attr[1];
-  const cudaLaunchConfig_t cfg = pair_config(1, nullptr, attr);
-  int clusters = 0;
-  e = cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_kernel<EPI, 256, false, false, true>,
-                                     &cfg);
-  if (e != cudaSuccess) return e;
-  if (clusters <= 0) return cudaErrorInvalidConfiguration;
-  if (g_max_pairs[device] == 0 || clusters < g_max_pairs[device]) g_max_pairs[device] = clusters;
-  return cudaSuccess;
-}
-
-int g_max_dual_pairs[kMaxDevices] = {0};
-
-cudaLaunchConfig_t dual_config(int pairs, cudaStream_t stream, cudaLaunchAttribute *attr) {
-  cudaLaunchConfig_t cfg = pair_config(pairs, stream, attr);
-  cfg.blockDim = dim3(kDualThreads, 1, 1);
-  cfg.dynamicSmemBytes = kDualSmemBytes;
   return cfg;
 }
 
@@ -1300,8 +1216,6 @@ cudaError_t gemm_prepare(int device) {
   cudaError_t e;
   if ((e = prepare_dual<kEpiSwiGLU>(device)) != cudaSuccess) return e;
   if ((e = prepare_dual<kEpiGated>(device)) != cudaSuccess) return e;
-  if ((e = prepare_pair<kEpiSwiGLU>(device)) != cudaSuccess) return e;
-  if ((e = prepare_pair<kEpiGated>(device)) != cudaSuccess) return e;
   if ((e = set_smem_limit<kEpiSwiGLU, 128>()) != cudaSuccess) return e;
   if ((e = set_smem_limit<kEpiGated, 128>()) != cudaSuccess) return e;
   if ((e = set_smem_limit<kEpiF32, 128>()) != cudaSuccess) return e;
@@ -1325,10 +1239,6 @@ int gemm_tile_tokens(long long rows, int groups, int K) {
   return (rows >= 128ll * groups && K >= 4096) ? 256 : 128;
 }
 
-int gemm_max_pairs(int device) {
-  return (device >= 0 && device < kMaxDevices) ? g_max_pairs[device] : 0;
-}
-
 int gemm_max_dual_pairs(int device) {
   return (device >= 0 && device < kMaxDevices) ? g_max_dual_pairs[device] : 0;
 }
@@ -1348,24 +1258,6 @@ cudaError_t launch_grouped_gemm_dual(int epi, const GemmArgs &args_in, int pairs
     case kEpiSwiGLU: return cudaLaunchKernelEx(&cfg, dual_gemm_kernel<kEpiSwiGLU>, args);
     case kEpiGated: return cudaLaunchKernelEx(&cfg, dual_gemm_kernel<kEpiGated>, args);
     default: return cudaErrorInvalidValue;
-  }
-}
-
-cudaError_t launch_grouped_gemm_pair(int epi, const GemmArgs &args_in, int pairs,
-                                     cudaStream_t stream) {
-  if (pairs <= 0) return cudaErrorInvalidConfiguration;
-  const GemmArgs args = with_limit(args_in);
-  cudaLaunchAttribute attr[1];
-  const cudaLaunchConfig_t cfg = pair_config(pairs, stream, attr);
-  switch (epi) {
-    case kEpiSwiGLU:
-      return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kEpiSwiGLU, 256, false, false, true>,
-                                args);
-    case kEpiGated:
-      return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kEpiGated, 256, false, false, true>,
-                                args);
-    default:
-      return cudaErrorInvalidValue;
   }
 }
 

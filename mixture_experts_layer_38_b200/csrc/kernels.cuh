@@ -69,19 +69,14 @@ void gemm_set_wait_limit(long long cycles);
 int gemm_tile_tokens(long long rows, int groups, int K);
 cudaError_t launch_grouped_gemm(int epi, const GemmArgs &args, int grid, int tile_tokens,
                                 cudaStream_t stream);
-// SwiGLU or gated grouped GEMM with 256-token tiles on CTA pairs (clusters of two SMs, pair
-// MMAs of 256 weight rows).  Needs M a multiple of 256 (SwiGLU) or 512 (gated); `pairs` = the
-// persistent pairs to launch (gemm_max_pairs caps it).
-cudaError_t launch_grouped_gemm_pair(int epi, const GemmArgs &args, int pairs,
-                                     cudaStream_t stream);
-int gemm_max_pairs(int device);  // co-resident pairs on the device (gemm_prepare queries it)
-// SwiGLU or gated grouped GEMM on CTA pairs running two pipelines per pair at once: full
-// 192-token tiles (and tails over 64 rows) beside tails of at most 64 rows, so tensor work and
-// weight streaming overlap within each SM.  Same M / K requirements as the pair launch; the
-// groups' row counts must satisfy gemm_dual_fits.
+// SwiGLU or gated grouped GEMM on CTA pairs (clusters of two SMs, pair MMAs of 256 weight
+// rows) running two pipelines per pair at once: full 192-token tiles (and tails over 64 rows)
+// beside tails of at most 64 rows, so tensor work and weight streaming overlap within each SM.
+// Needs M a multiple of 256 (SwiGLU) or 512 (gated), group row counts within gemm_dual_fits;
+// `pairs` = the persistent pairs to launch (gemm_max_dual_pairs caps it).
 cudaError_t launch_grouped_gemm_dual(int epi, const GemmArgs &args, int pairs,
                                      cudaStream_t stream);
-int gemm_max_dual_pairs(int device);
+int gemm_max_dual_pairs(int device);  // co-resident pairs on the device (gemm_prepare queries it)
 bool gemm_dual_fits(long long rows, int groups);
 // SwiGLU or gated grouped GEMM with E4M3 block-quantised weights, 128-token tiles.
 cudaError_t launch_grouped_gemm_fp8(int epi, const GemmArgs &args, int grid,

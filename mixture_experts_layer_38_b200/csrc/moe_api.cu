@@ -25,8 +25,7 @@ struct DeviceInfo {
   bool ready = false;
   int status = MOE_OK;
   int sms = 0;
-  int pairs = 0;  // persistent CTA pairs of the pair GEMMs (co-resident, at most sms / 2)
-  int dual_pairs = 0;  // the same for the two-pipeline pair GEMMs
+  int dual_pairs = 0;  // persistent CTA pairs of the pair GEMMs (co-resident, <= sms / 2)
 };
 
 std::mutex g_mu;
@@ -52,7 +51,6 @@ int device_info(const DeviceInfo **out) {
       di.status = MOE_OK;
     }
     di.sms = sms;
-    di.pairs = di.status == MOE_OK ? std::min(gemm_max_pairs(dev), sms / 2) : 0;
     di.dual_pairs = di.status == MOE_OK ? std::min(gemm_max_dual_pairs(dev), sms / 2) : 0;
     di.ready = true;
   }
@@ -315,11 +313,11 @@ int do_expert_ffn(const moe_dims &d, const DeviceInfo &di, const Layout &L,
   const bool gather = perm_tok != nullptr;
   const int tile_tokens = gemm_tile_tokens((long long)rows, d.N, d.d);
   const bool p256 = fw != nullptr || tile_tokens != 256;  // L2 promotion, see make_map
-  // 256-token tiles run on CTA pairs where the weight rows split into whole pair tiles.
-  const bool pair = fw == nullptr && !gather && tile_tokens == 256 && di.pairs > 0 &&
-                    d.I % 256 == 0 && d.d % 512 == 0;
-  // On CTA pairs the two-pipeline kernel runs full and tail tiles side by side.
-  const bool dual = pair && di.dual_pairs > 0 && gemm_dual_fits((long long)rows, d.N);
+  // Wide tiles run on CTA pairs (two pipelines per pair: full and tail tiles side by side)
+  // where the weight rows split into whole pair tiles; otherwise on single CTAs.
+  const bool dual = fw == nullptr && !gather && tile_tokens == 256 && di.dual_pairs > 0 &&
+                    d.I % 256 == 0 && d.d % 512 == 0 &&
+                    gemm_dual_fits((long long)rows, d.N);
   const bool ok_w = fw != nullptr
       ? make_map_u8(&up.map_a0, fw->q_g, (uint64_t)d.N * d.I, (uint64_t)d.d) &&
             make_map_u8(&up.map_a1, fw->q_u, (uint64_t)d.N * d.I, (uint64_t)d.d) &&
@@ -355,7 +353,6 @@ int do_expert_ffn(const moe_dims &d, const DeviceInfo &di, const Layout &L,
   }
   if ((fw != nullptr ? launch_grouped_gemm_fp8(kEpiSwiGLU, up, di.sms, stream)
        : dual        ? launch_grouped_gemm_dual(kEpiSwiGLU, up, di.dual_pairs, stream)
-       : pair        ? launch_grouped_gemm_pair(kEpiSwiGLU, up, di.pairs, stream)
                      : launch_grouped_gemm(kEpiSwiGLU, up, di.sms, tile_tokens, stream)) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
@@ -392,7 +389,6 @@ int do_expert_ffn(const moe_dims &d, const DeviceInfo &di, const Layout &L,
     return to_status(launch_grouped_gemm_fp8(kEpiGated, down, di.sms, stream));
   }
   if (dual) return to_status(launch_grouped_gemm_dual(kEpiGated, down, di.dual_pairs, stream));
-  if (pair) return to_status(launch_grouped_gemm_pair(kEpiGated, down, di.pairs, stream));
   return to_status(launch_grouped_gemm(kEpiGated, down, di.sms, tile_tokens, stream));
 }
 

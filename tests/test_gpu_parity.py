@@ -118,6 +118,7 @@ def test_expert_ffn_matches_oracle(name):
     (512, (520, 300, 256, 100, 17, 1, 0, 30)),
     (384, (520, 300, 256, 100, 17, 1, 0, 30)),
     (512, (192, 193, 65, 64, 384, 257, 0, 129)),
+    (512, (224, 225, 33, 32, 448, 256, 0, 130)),
 ])
 def test_expert_ffn_wide_tiles_matches_oracle(I, counts):
     # d = 4096 with >= 128 rows per expert selects the wide tiles: I = 512 runs them on CTA
@@ -125,9 +126,10 @@ def test_expert_ffn_wide_tiles_matches_oracle(I, counts):
     # and tails over 64 rows in one pipeline, tails of at most 64 rows in the other), I = 384
     # on single CTAs with 256-token tiles.  Ragged groups built directly: several full tiles
     # with and without tails, tail-only experts (100 / 30 / 17 / 1 rows), an empty expert; the
-    # third case sits on the two-pipeline kernel's boundaries (192 = one full tile, 193 = one
-    # full tile + a 1-row tail, 65 = the smallest tail kept in the full-tile pipeline, 64 = the
-    # largest in the tail pipeline, 384, 257 = 192 + 65, 129).  Rows = K = 4 times the tokens.
+    # last case sits on the two-pipeline kernel's boundaries (224-row full tiles, tails of at
+    # most 32 rows in the tail pipeline): 224 = one full tile, 225 = one full tile + a 1-row
+    # tail, 33 = the smallest remainder kept in the full-tile pipeline, 32 = the largest in the
+    # tail pipeline, 448, 256 = 224 + 32, 130.  Rows = K = 4 times the tokens.
     counts = np.array(counts)
     R = int(counts.sum())
     w = Workload("wide", T=R // 4, d=4096, N=8, Z=4, K=4, I=I)
