@@ -20,9 +20,8 @@
 // holding half the weight rows and half the token rows of a stage, and each pair runs two
 // pipelines at once, full tiles beside the lightly used experts' weight-streaming tails.
 //
-// Warp roles (64 + 32 x kGemmEpiWarps = 192 threads, one CTA per SM, persistent over a static
-// tile schedule; with CTA pairs only the even CTA's warp 1 issues MMAs, whose commits signal
-// both CTAs, and both CTAs' epilogues release the accumulator on the even CTA's barrier):
+// Warp roles of the single-CTA kernel (64 + 32 x kGemmEpiWarps = 192 threads, one CTA per SM,
+// persistent over a static tile schedule; the two-pipeline pair kernel has two such sets):
 //   warp 0      TMA producer: A0/A1 weight tiles (128 x 64) and the token tile (n x 64, issued
 //               as 256/128/64/32/16-row boxes) into a 192 KB ring of 48 KB or 64 KB stages
 //   warp 1      TMEM allocator (512 columns: 2 buffers x 2 x 128, or 1 x 2 x 256) and MMA issuer
@@ -748,30 +747,38 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER>::kThreads, 1)
 // ==================================================================== dual-pipeline CTA pairs
 // Each CTA pair runs two independent pipelines at once, each with its own shared-memory ring,
 // barriers, TMA producer, MMA issuer, four epilogue warps and TMEM columns:
-//   F  full token tiles of kDualBNF = 192 rows, and the tail of an expert when it holds more than
-//      kDualBNL rows (compute-bound: 3 stages of 2 x 16 KB weights + 96 token rows per CTA,
-//      2 x 192 accumulator columns);
-//   L  an expert's tail of at most kDualBNL = 64 rows (weight streaming: 2 stages of 2 x 16 KB
-//      weights + 32 token rows per CTA, 2 x 64 accumulator columns).
+//   F  full token tiles of kDualBNF = 224 rows, and the tail of an expert when it holds more than
+//      kDualBNL rows (compute-bound: 3 stages of 2 x 16 KB weights + 112 token rows per CTA,
+//      2 x 224 accumulator columns);
+//   L  an expert's tail of at most kDualBNL = 32 rows (weight streaming: 2 stages of 2 x 16 KB
+//      weights + 16 token rows per CTA, 2 x 32 accumulator columns).
 // With one pipeline per SM every SM alternated between streaming a lightly used expert's weights
 // (tensor pipe idle) and a heavily used expert's compute-bound tiles; here both kinds of tile are
 // in flight on every SM, so HBM streaming and tensor work overlap within each SM.  Items of each
 // list are dealt round-robin over the pairs; within a token tile the weight tiles come fastest.
-constexpr int kDualBNF = 192;
-constexpr int kDualBNL = 64;
+constexpr int kDualBNF = 224;
+constexpr int kDualBNL = 32;
 constexpr int kDualStagesF = 3;
 constexpr int kDualStagesL = 2;
-constexpr int kDualStageF = 2 * kTileA + (kDualBNF / 2) * kBK * 2;  // 44 KB
-constexpr int kDualStageL = 2 * kTileA + (kDualBNL / 2) * kBK * 2;  // 36 KB
+constexpr int kDualStageF = 2 * kTileA + (kDualBNF / 2) * kBK * 2;  // 46 KB
+constexpr int kDualStageL = 2 * kTileA + (kDualBNL / 2) * kBK * 2;  // 34 KB
 constexpr int kDualEpiWarps = 4;                                     // per pipeline
 constexpr int kDualThreads = 32 * 2 * (2 + kDualEpiWarps);           // 384
 constexpr int kDualRing = kDualStagesF * kDualStageF + kDualStagesL * kDualStageL;
 constexpr int kDualStaging = 2 * kDualEpiWarps * kStagingFloats * 4;
-constexpr int kDualPrefix = 2 * (kMaxGroups + 4) * 2;               // uint16 prefixes
+// uint16 prefixes of F and L tiles per group, sized per launch for the groups present (the
+// maximum group count does not fit beside the rings).
+__host__ __device__ constexpr int dual_prefix_len(int groups) { return (groups + 4 + 7) & ~7; }
 constexpr int kDualBarsPerPipe = 2 * kDualStagesF + 3;
-constexpr int kDualSmemBytes = 1024 + kDualRing + kDualStaging + kDualPrefix +
-                               2 * kDualBarsPerPipe * 8 + 16;
-static_assert(kDualSmemBytes <= 232448, "shared memory per block");
+constexpr int kDualSmemFixed = 1024 + kDualRing + kDualStaging + 2 * kDualBarsPerPipe * 8 + 16;
+constexpr int kDualSmemLimit = 232448;  // shared memory per block
+__host__ __device__ constexpr int dual_smem_bytes(int groups) {
+  return kDualSmemFixed + 2 * dual_prefix_len(groups) * 2;
+}
+static_assert(kDualStageF % 1024 == 0 && kDualStageL % 1024 == 0, "1024-byte-aligned stages");
+// Most groups whose prefixes fit: 512 + 256 experts need 512.
+constexpr int kDualMaxGroups = 960;
+static_assert(dual_smem_bytes(kDualMaxGroups) <= kDualSmemLimit, "shared memory per block");
 static_assert(2 * kDualBNF + 2 * kDualBNL <= kTmemCols, "TMEM holds 512 columns");
 
 struct DualSchedule {
@@ -1032,8 +1039,9 @@ __global__ void __launch_bounds__(kDualThreads, 1)
   uint8_t *ring_l = smem + kDualStagesF * kDualStageF;
   float *staging = reinterpret_cast<float *>(smem + kDualRing);
   uint16_t *fpre = reinterpret_cast<uint16_t *>(smem + kDualRing + kDualStaging);
-  uint16_t *lpre = fpre + kMaxGroups + 4;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kDualRing + kDualStaging + kDualPrefix);
+  const int pfx = dual_prefix_len(args.num_groups);
+  uint16_t *lpre = fpre + pfx;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kDualRing + kDualStaging + 2 * pfx * 2);
   // per pipeline p: full[kDualStagesF], empty[kDualStagesF], tfull, tempty, drain
   uint64_t *bf = bars, *bl = bars + kDualBarsPerPipe;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * kDualBarsPerPipe);
@@ -1154,11 +1162,12 @@ constexpr int kMaxDevices = 64;
 int g_max_dual_pairs[kMaxDevices] = {0};
 
 // Clusters of two CTAs (one CTA pair per cluster) of the two-pipeline kernel.
-cudaLaunchConfig_t dual_config(int pairs, cudaStream_t stream, cudaLaunchAttribute *attr) {
+cudaLaunchConfig_t dual_config(int pairs, int groups, cudaStream_t stream,
+                               cudaLaunchAttribute *attr) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
   cfg.blockDim = dim3(kDualThreads, 1, 1);
-  cfg.dynamicSmemBytes = kDualSmemBytes;
+  cfg.dynamicSmemBytes = dual_smem_bytes(groups);
   cfg.stream = stream;
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
@@ -1173,10 +1182,10 @@ template <int EPI>
 cudaError_t prepare_dual(int device) {
   cudaError_t e = cudaFuncSetAttribute(dual_gemm_kernel<EPI>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       kDualSmemBytes);
+                                       kDualSmemLimit);
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr[1];
-  const cudaLaunchConfig_t cfg = dual_config(1, nullptr, attr);
+  const cudaLaunchConfig_t cfg = dual_config(1, kDualMaxGroups, nullptr, attr);
   int clusters = 0;
   e = cudaOccupancyMaxActiveClusters(&clusters, dual_gemm_kernel<EPI>, &cfg);
   if (e != cudaSuccess) return e;
@@ -1244,8 +1253,9 @@ int gemm_max_dual_pairs(int device) {
 }
 
 bool gemm_dual_fits(long long rows, int groups) {
-  // Per-group tile prefixes are 16-bit: F tiles <= rows / 192 + groups, L tiles <= groups.
-  return groups <= kMaxGroups && rows / kDualBNF + groups + 8 < 65536;
+  // Per-group tile prefixes are 16-bit (F tiles <= rows / BNF + groups, L tiles <= groups) and
+  // sized to the groups present, within the shared memory beside the rings.
+  return groups <= kDualMaxGroups && rows / kDualBNF + groups + 8 < 65536;
 }
 
 cudaError_t launch_grouped_gemm_dual(int epi, const GemmArgs &args_in, int pairs,
@@ -1253,7 +1263,7 @@ cudaError_t launch_grouped_gemm_dual(int epi, const GemmArgs &args_in, int pairs
   if (pairs <= 0) return cudaErrorInvalidConfiguration;
   const GemmArgs args = with_limit(args_in);
   cudaLaunchAttribute attr[1];
-  const cudaLaunchConfig_t cfg = dual_config(pairs, stream, attr);
+  const cudaLaunchConfig_t cfg = dual_config(pairs, args.num_groups, stream, attr);
   switch (epi) {
     case kEpiSwiGLU: return cudaLaunchKernelEx(&cfg, dual_gemm_kernel<kEpiSwiGLU>, args);
     case kEpiGated: return cudaLaunchKernelEx(&cfg, dual_gemm_kernel<kEpiGated>, args);
