@@ -49,8 +49,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # while the kernel and its launch set-up are unchanged (sha1 of the code, comments removed, of
 # the GEMM kernel and of the file that builds its tensor maps, at capture time).
 NCU_TRAFFIC = {
-    ("prefill", "ffn_up_gemm"): {"bytes_per_launch": 36312271360, "src": "a1a46c489207"},
-    ("decode", "ffn_up_gemm"): {"bytes_per_launch": 7316081920, "src": "a1a46c489207"},
+    ("prefill", "ffn_up_gemm"): {"bytes_per_launch": 41377593600, "src": "5a35ac00afb5"},
+    ("prefill", "ffn_down_gemm"): {"bytes_per_launch": 17432248064, "src": "5a35ac00afb5"},
+    ("decode", "ffn_up_gemm"): {"bytes_per_launch": 7316193024, "src": "5a35ac00afb5"},
 }
 
 
