@@ -52,9 +52,14 @@ def _load():
         _lib.oracle_dequantize_fp8_blocks.argtypes = [_i64, _i64, _i64, _ptr, _ptr, _ptr]
         _lib.oracle_dequantize_fp8_blocks.restype = None
         _lib.oracle_balance_step.argtypes = [_i64, _ptr, _ptr, ctypes.c_float]
+        _lib.oracle_quantize_fp8_rows.argtypes = [_i64, _i64, _ptr, _ptr, _ptr]
+        _lib.oracle_swiglu_expert_fp8act.argtypes = list(_lib.oracle_swiglu_expert.argtypes)
+        _lib.oracle_combine_tokens_fp8act.argtypes = list(_lib.oracle_combine_tokens.argtypes)
         for f in ("oracle_router", "oracle_dispatch", "oracle_swiglu_expert",
                   "oracle_combine_tokens", "oracle_combine_rows", "oracle_forward",
-                  "oracle_pid_step", "oracle_renormalize_gates", "oracle_balance_step"):
+                  "oracle_pid_step", "oracle_renormalize_gates", "oracle_balance_step",
+                  "oracle_quantize_fp8_rows", "oracle_swiglu_expert_fp8act",
+                  "oracle_combine_tokens_fp8act"):
             getattr(_lib, f).restype = None
     return _lib
 
@@ -143,20 +148,28 @@ def dispatch(topk_idx, N, E):
     return {"counts": counts, "offsets": offsets, "perm_tok": perm_tok[:A], "slot_pos": slot_pos}
 
 
-def swiglu_expert(xrows, W_g, W_u, W_d):
-    """E(x) = W_d (silu(W_g x) * (W_u x)) for each row of xrows, in fp64."""
+def swiglu_expert(xrows, W_g, W_u, W_d, fp8_act=False):
+    """E(x) = W_d (silu(W_g x) * (W_u x)) for each row of xrows, in fp64.
+
+    With ``fp8_act`` the token rows and h are quantised to E4M3 in 1 x 128 blocks (see
+    :func:`quantize_fp8_rows`) before the products; d and I must be multiples of 128."""
     xrows, W_g, W_u, W_d = bf16_bits(xrows), bf16_bits(W_g), bf16_bits(W_u), bf16_bits(W_d)
     R, d = xrows.shape
     I = W_g.shape[0]
     assert W_g.shape == (I, d) and W_u.shape == (I, d) and W_d.shape == (d, I)
+    if fp8_act:
+        assert d % 128 == 0 and I % 128 == 0
     out = np.zeros((R, d), np.float64)
     if R:
-        _load().oracle_swiglu_expert(d, I, R, _p(xrows), _p(W_g), _p(W_u), _p(W_d), _p(out))
+        fn = _load().oracle_swiglu_expert_fp8act if fp8_act else _load().oracle_swiglu_expert
+        fn(d, I, R, _p(xrows), _p(W_g), _p(W_u), _p(W_d), _p(out))
     return out
 
 
-def combine_tokens(tokens, x, topk_idx, topk_gate, W_g, W_u, W_d, N):
-    """y_t = sum_k g_{t,k} E_{i_{t,k}}(x_t) for the listed tokens (weights all in host memory)."""
+def combine_tokens(tokens, x, topk_idx, topk_gate, W_g, W_u, W_d, N, fp8_act=False):
+    """y_t = sum_k g_{t,k} E_{i_{t,k}}(x_t) for the listed tokens (weights all in host memory).
+
+    ``fp8_act``: the FFN experts quantise their activations (see :func:`swiglu_expert`)."""
     x, W_g, W_u, W_d = bf16_bits(x), bf16_bits(W_g), bf16_bits(W_u), bf16_bits(W_d)
     topk_idx = _i32(topk_idx)
     topk_gate = np.ascontiguousarray(topk_gate, dtype=np.float64)
@@ -164,9 +177,12 @@ def combine_tokens(tokens, x, topk_idx, topk_gate, W_g, W_u, W_d, N):
     T, d = x.shape
     K = topk_idx.shape[1]
     I = W_g.shape[1]
+    if fp8_act:
+        assert d % 128 == 0 and I % 128 == 0
     y = np.zeros((len(tokens), d), np.float64)
-    _load().oracle_combine_tokens(d, N, K, I, len(tokens), _p(tokens), _p(x), _p(topk_idx),
-                                  _p(topk_gate), _p(W_g), _p(W_u), _p(W_d), _p(y))
+    fn = _load().oracle_combine_tokens_fp8act if fp8_act else _load().oracle_combine_tokens
+    fn(d, N, K, I, len(tokens), _p(tokens), _p(x), _p(topk_idx), _p(topk_gate), _p(W_g),
+       _p(W_u), _p(W_d), _p(y))
     return y
 
 
@@ -209,14 +225,15 @@ def forward(x, W_r, b, W_g, W_u, W_d, N, Z, K, renormalize=False):
     return {"y": y, "topk_idx": idx, "topk_gate": gate, "gap": gap}
 
 
-def forward_sampled(tokens, x, W_r, b, N, Z, K, fetch_expert, routing=None):
+def forward_sampled(tokens, x, W_r, b, N, Z, K, fetch_expert, routing=None, fp8_act=False):
     """The layer's output for a sample of tokens when the weights live elsewhere.
 
     ``fetch_expert(i)`` returns (W_g[i], W_u[i], W_d[i]) as bf16 arrays ([I,d], [I,d], [d,I]).
     Routing (router + biased top-K) is computed here for the sampled rows unless ``routing``
     (a dict like :func:`router`'s, for exactly these rows) is given.  Each distinct FFN expert
     is fetched once and applied to all sampled rows that selected it; the K slot terms of each
-    token are then summed in slot order, as in oracle_combine_tokens.
+    token are then summed in slot order, as in oracle_combine_tokens.  ``fp8_act`` as in
+    :func:`swiglu_expert`.
     """
     tokens = np.asarray(tokens, dtype=np.int64)
     xs = bf16_bits(x)[tokens] if not hasattr(x, "detach") else bf16_bits(x[tokens])
@@ -232,7 +249,7 @@ def forward_sampled(tokens, x, W_r, b, N, Z, K, fetch_expert, routing=None):
     for i in np.unique(idx[idx < N]):
         rows, slots = np.nonzero(idx == i)
         W_g, W_u, W_d = fetch_expert(int(i))
-        terms[rows, slots, :] = swiglu_expert(xs[rows], W_g, W_u, W_d)
+        terms[rows, slots, :] = swiglu_expert(xs[rows], W_g, W_u, W_d, fp8_act=fp8_act)
     y = np.zeros((n, d), np.float64)
     for k in range(K):
         y += gate[:, k:k + 1] * terms[:, k, :]
@@ -291,3 +308,20 @@ def dequantize_fp8_blocks(q, scale):
     w = np.zeros((G, R, C), np.uint16)
     _load().oracle_dequantize_fp8_blocks(G, R, C, _p(q), _p(scale), _p(w))
     return w
+
+
+def quantize_fp8_rows(v):
+    """FP8 activations: rows of v [R, C] (C a multiple of 128; float values, fp64 exact) ->
+    (q uint8 [R, C], scale float32 [R, C/128]), one power-of-two scale per 1 x 128 block by
+    the weights' rule (smallest 2^e with max|v| <= 448 * 2^e, e >= -126, 1 for an all-zero
+    block; q = E4M3(v / 2^e), nearest, ties to even)."""
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    if v.ndim == 1:
+        v = v[None]
+    R, C = v.shape
+    assert C % 128 == 0
+    q = np.zeros((R, C), np.uint8)
+    scale = np.zeros((R, C // 128), np.float32)
+    if R and C:
+        _load().oracle_quantize_fp8_rows(R, C, _p(v), _p(q), _p(scale))
+    return q, scale

@@ -163,6 +163,8 @@ void oracle_dispatch(int64_t T, int64_t K, int64_t N, int64_t E, const int32_t *
     free(cursor);
 }
 
+static void fp8_round_trip_row(int64_t n, double *v);
+
 /* ------------------------------------------------------------------------------------------
  * One FFN expert on R input rows (P1 §零計算專家 calls them standard FFN experts; the
  * SwiGLU form is the reading taken here):
@@ -192,16 +194,65 @@ static void swiglu_row(int64_t d, int64_t I, const uint16_t *xr, const uint16_t 
     }
 }
 
-void oracle_swiglu_expert(int64_t d, int64_t I, int64_t R, const uint16_t *xrows,
-                          const uint16_t *W_g, const uint16_t *W_u, const uint16_t *W_d,
-                          double *out)
+/* The same expert with FP8 activations (an optional variant, used with FP8 weights; see the
+ * FP8 section below): the token row is quantised in 1 x 128 blocks and the values q * 2^e enter
+ * the up-projection; h is quantised the same way before the down projection.  Everything else
+ * is as in swiglu_row, in fp64.  xv holds d doubles of scratch. */
+static void swiglu_row_fp8act(int64_t d, int64_t I, const uint16_t *xr, const uint16_t *W_g,
+                              const uint16_t *W_u, const uint16_t *W_d, double *xv, double *h,
+                              double *out)
+{
+    for (int64_t j = 0; j < d; ++j) xv[j] = bf16_to_f64(xr[j]);
+    fp8_round_trip_row(d, xv);
+    for (int64_t f = 0; f < I; ++f) {
+        double a = 0.0, u = 0.0;
+        const uint16_t *wg = W_g + f * d;
+        const uint16_t *wu = W_u + f * d;
+        for (int64_t j = 0; j < d; ++j) {
+            a += bf16_to_f64(wg[j]) * xv[j];
+            u += bf16_to_f64(wu[j]) * xv[j];
+        }
+        h[f] = (a / (1.0 + exp(-a))) * u;
+    }
+    fp8_round_trip_row(I, h);
+    for (int64_t j = 0; j < d; ++j) {
+        const uint16_t *wd = W_d + j * I;
+        double acc = 0.0;
+        for (int64_t f = 0; f < I; ++f) acc += bf16_to_f64(wd[f]) * h[f];
+        out[j] = acc;
+    }
+}
+
+static void expert_rows(int64_t d, int64_t I, int64_t R, const uint16_t *xrows,
+                        const uint16_t *W_g, const uint16_t *W_u, const uint16_t *W_d,
+                        double *out, int fp8act)
 {
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t r = 0; r < R; ++r) {
         double *h = (double *)malloc(sizeof(double) * (size_t)I);
-        swiglu_row(d, I, xrows + r * d, W_g, W_u, W_d, h, out + r * d);
+        double *xv = (double *)malloc(sizeof(double) * (size_t)d);
+        if (fp8act)
+            swiglu_row_fp8act(d, I, xrows + r * d, W_g, W_u, W_d, xv, h, out + r * d);
+        else
+            swiglu_row(d, I, xrows + r * d, W_g, W_u, W_d, h, out + r * d);
+        free(xv);
         free(h);
     }
+}
+
+void oracle_swiglu_expert(int64_t d, int64_t I, int64_t R, const uint16_t *xrows,
+                          const uint16_t *W_g, const uint16_t *W_u, const uint16_t *W_d,
+                          double *out)
+{
+    expert_rows(d, I, R, xrows, W_g, W_u, W_d, out, 0);
+}
+
+/* d and I multiples of 128. */
+void oracle_swiglu_expert_fp8act(int64_t d, int64_t I, int64_t R, const uint16_t *xrows,
+                                 const uint16_t *W_g, const uint16_t *W_u, const uint16_t *W_d,
+                                 double *out)
+{
+    expert_rows(d, I, R, xrows, W_g, W_u, W_d, out, 1);
 }
 
 /* ------------------------------------------------------------------------------------------
@@ -211,15 +262,16 @@ void oracle_swiglu_expert(int64_t d, int64_t I, int64_t R, const uint16_t *xrows
  * Weights are the natural per-expert layouts: W_g, W_u [N][I][d]; W_d [N][d][I].
  * Only tokens listed in `tokens` (n_tok of them) are computed; y has n_tok rows.
  * ---------------------------------------------------------------------------------------- */
-void oracle_combine_tokens(int64_t d, int64_t N, int64_t K, int64_t I, int64_t n_tok,
+static void combine_tokens(int64_t d, int64_t N, int64_t K, int64_t I, int64_t n_tok,
                            const int64_t *tokens, const uint16_t *x, const int32_t *topk_idx,
                            const double *topk_gate, const uint16_t *W_g, const uint16_t *W_u,
-                           const uint16_t *W_d, double *y)
+                           const uint16_t *W_d, double *y, int fp8act)
 {
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t n = 0; n < n_tok; ++n) {
         double *h = (double *)malloc(sizeof(double) * (size_t)I);
         double *ffn = (double *)malloc(sizeof(double) * (size_t)d);
+        double *xv = (double *)malloc(sizeof(double) * (size_t)d);
         int64_t t = tokens[n];
         const uint16_t *xt = x + t * d;
         double *yt = y + n * d;
@@ -229,15 +281,39 @@ void oracle_combine_tokens(int64_t d, int64_t N, int64_t K, int64_t I, int64_t n
             double g = topk_gate[t * K + k];
             if (i >= N) { /* zero-computation expert: E_i(x) = x */
                 for (int64_t j = 0; j < d; ++j) yt[j] += g * bf16_to_f64(xt[j]);
+            } else if (fp8act) {
+                swiglu_row_fp8act(d, I, xt, W_g + (int64_t)i * I * d, W_u + (int64_t)i * I * d,
+                                  W_d + (int64_t)i * d * I, xv, h, ffn);
+                for (int64_t j = 0; j < d; ++j) yt[j] += g * ffn[j];
             } else {
                 swiglu_row(d, I, xt, W_g + (int64_t)i * I * d, W_u + (int64_t)i * I * d,
                            W_d + (int64_t)i * d * I, h, ffn);
                 for (int64_t j = 0; j < d; ++j) yt[j] += g * ffn[j];
             }
         }
+        free(xv);
         free(h);
         free(ffn);
     }
+}
+
+void oracle_combine_tokens(int64_t d, int64_t N, int64_t K, int64_t I, int64_t n_tok,
+                           const int64_t *tokens, const uint16_t *x, const int32_t *topk_idx,
+                           const double *topk_gate, const uint16_t *W_g, const uint16_t *W_u,
+                           const uint16_t *W_d, double *y)
+{
+    combine_tokens(d, N, K, I, n_tok, tokens, x, topk_idx, topk_gate, W_g, W_u, W_d, y, 0);
+}
+
+/* The same with FP8 activations in the FFN experts (zero experts still return x_t unchanged:
+ * no product, nothing to quantise).  d and I multiples of 128. */
+void oracle_combine_tokens_fp8act(int64_t d, int64_t N, int64_t K, int64_t I, int64_t n_tok,
+                                  const int64_t *tokens, const uint16_t *x,
+                                  const int32_t *topk_idx, const double *topk_gate,
+                                  const uint16_t *W_g, const uint16_t *W_u, const uint16_t *W_d,
+                                  double *y)
+{
+    combine_tokens(d, N, K, I, n_tok, tokens, x, topk_idx, topk_gate, W_g, W_u, W_d, y, 1);
 }
 
 /* ------------------------------------------------------------------------------------------
@@ -367,7 +443,11 @@ void oracle_balance_step(int64_t N, const int32_t *counts, float *b, float gamma
  * no infinities; S.1111.111 is NaN; largest finite 448); each block's scale is the smallest
  * power of two 2^e with max|w| <= 448 * 2^e (a power of two keeps q * 2^e exact in bf16);
  * q = E4M3(w / 2^e) rounded to nearest, ties to even mantissa, saturating at +-448.
- * Activations stay bf16 (weight-only quantisation).
+ * By default activations stay bf16 (weight-only quantisation).  The FP8-activation variant
+ * quantises the inputs of both expert GEMMs too -- the token row x_t and h -- at the activation
+ * granularity of the DeepSeek-V3 scheme the page names: one scale per token per 128 consecutive
+ * channels (a 1 x 128 block), with the same format and scale rule (reading: the page names the
+ * scheme only).
  * ---------------------------------------------------------------------------------------- */
 double oracle_e4m3_decode(uint8_t code)
 {
@@ -393,6 +473,20 @@ uint8_t oracle_e4m3_encode(double v)
     double mq = nearbyint((ldexp(a, -e) - 1.0) * 8.0);
     if (mq == 8.0) { mq = 0.0; e += 1; }
     return (uint8_t)(s | (uint8_t)(((e + 7) << 3) | (int)mq));
+}
+
+/* The exponent e of a block's scale 2^e: the smallest integer with amax <= 448 * 2^e, at least
+ * -126; 0 for an all-zero block. */
+static int fp8_scale_exponent(double amax)
+{
+    int e = 0;
+    if (amax > 0.0) {
+        e = ilogb(amax) - 8;
+        while (amax > ldexp(448.0, e)) ++e;
+        while (amax <= ldexp(448.0, e - 1)) --e;
+        if (e < -126) e = -126;
+    }
+    return e;
 }
 
 /* Round-to-nearest-even conversion of a double that is exact in fp32 to bf16 bits. */
@@ -422,13 +516,7 @@ void oracle_quantize_fp8_blocks(int64_t G, int64_t R, int64_t C, const uint16_t 
                     const double a = fabs(bf16_to_f64(w[(g * R + rb * 128 + r) * C + cb * 128 + c]));
                     if (a > amax) amax = a;
                 }
-            int e = 0;
-            if (amax > 0.0) {
-                e = ilogb(amax) - 8;
-                while (amax > ldexp(448.0, e)) ++e;
-                while (amax <= ldexp(448.0, e - 1)) --e;
-                if (e < -126) e = -126;
-            }
+            const int e = fp8_scale_exponent(amax);
             scale[(g * RB + rb) * CB + cb] = (float)ldexp(1.0, e);
             for (int64_t r = 0; r < 128; ++r)
                 for (int64_t c = 0; c < 128; ++c) {
@@ -452,4 +540,33 @@ void oracle_dequantize_fp8_blocks(int64_t G, int64_t R, int64_t C, const uint8_t
                 const double s = (double)scale[(g * RB + r / 128) * CB + c / 128];
                 w[i] = f64_to_bf16_rne(oracle_e4m3_decode(q[i]) * s);
             }
+}
+
+/* FP8 activations: v [R][C] (C a multiple of 128) -> q [R][C] E4M3 codes and scale
+ * [R][C/128] fp32 (= 2^e), one scale per 1 x 128 block of a row, by the weights' rule. */
+void oracle_quantize_fp8_rows(int64_t R, int64_t C, const double *v, uint8_t *q, float *scale)
+{
+    const int64_t CB = C / 128;
+    for (int64_t r = 0; r < R; ++r)
+        for (int64_t cb = 0; cb < CB; ++cb) {
+            const double *blk = v + r * C + cb * 128;
+            double amax = 0.0;
+            for (int64_t c = 0; c < 128; ++c)
+                if (fabs(blk[c]) > amax) amax = fabs(blk[c]);
+            const int e = fp8_scale_exponent(amax);
+            scale[r * CB + cb] = (float)ldexp(1.0, e);
+            for (int64_t c = 0; c < 128; ++c)
+                q[r * C + cb * 128 + c] = oracle_e4m3_encode(ldexp(blk[c], -e));
+        }
+}
+
+/* v [n] (n a multiple of 128) replaced in place by its FP8-activation value q * 2^e. */
+static void fp8_round_trip_row(int64_t n, double *v)
+{
+    uint8_t *q = (uint8_t *)malloc((size_t)n);
+    float *s = (float *)malloc(sizeof(float) * (size_t)(n / 128 > 0 ? n / 128 : 1));
+    oracle_quantize_fp8_rows(1, n, v, q, s);
+    for (int64_t i = 0; i < n; ++i) v[i] = oracle_e4m3_decode(q[i]) * (double)s[i / 128];
+    free(s);
+    free(q);
 }
