@@ -77,7 +77,8 @@ def _code_only(text):
 
 def gemm_source_hash(read=None):
     h = hashlib.sha1()
-    for name in ("gemm.cu", "device.cuh", "kernels.cuh", "moe_api.cu"):
+    for name in ("gemm.cu", "gemm_common.cuh", "gemm_f8.cu", "device.cuh", "kernels.cuh",
+                 "moe_api.cu"):
         path = os.path.join("mixture_experts_layer_38_b200", "csrc", name)
         if read is None:
             with open(os.path.join(ROOT, path), encoding="utf-8") as f:
@@ -213,10 +214,12 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------ work model
-def work_model(w, counts, wb=2):
+def work_model(w, counts, wb=2, ab=2):
     """Algorithmic FLOPs and bytes of one step from the routing actually taken; `wb` bytes per
     expert weight (2 for bf16, 1 for the FP8 codes; their block scales add 4 bytes per 16384
-    weights, negligible)."""
+    weights, negligible), `ab` bytes per GEMM activation (2 for bf16, 1 for FP8 activations,
+    whose up-projection stage also holds the quantisation of x_perm: 2 bytes read, 1 written
+    per element; block scales again negligible)."""
     counts = np.asarray(counts, np.int64)
     A = int(counts[:w.N].sum())
     U = int((counts[:w.N] > 0).sum())
@@ -228,8 +231,9 @@ def work_model(w, counts, wb=2):
     }
     bytes_ = {
         "router_gemm": E * d * 2 + T * d * 2 + T * E * 4,
-        "ffn_up_gemm": U * 2 * I * d * wb + A * d * 2 + A * I * 2,
-        "ffn_down_gemm": U * d * I * wb + A * I * 2 + A * d * 2,
+        "ffn_up_gemm": U * 2 * I * d * wb + A * d * ab + A * I * ab +
+                       (A * d * 3 if ab == 1 else 0),
+        "ffn_down_gemm": U * d * I * wb + A * I * ab + A * d * 2,
         "dispatch": 2 * A * d * 2,
         "combine": (A + 2 * T) * d * 2,
     }
@@ -245,14 +249,14 @@ def stage_durations(events):
     return stage_ms
 
 
-def step_work(w, hist, wb=2):
+def step_work(w, hist, wb=2, ab=2):
     """Algorithmic FLOPs and bytes summed over the steps whose per-expert counts are `hist`."""
     tot_flops = {k: 0 for k in ("router_gemm", "ffn_up_gemm", "ffn_down_gemm")}
     tot_bytes = {k: 0 for k in ("router_gemm", "ffn_up_gemm", "ffn_down_gemm", "dispatch",
                                 "combine")}
     A_steps, U_steps, load_ratio = [], [], []
     for c in hist:
-        A, U, fl, by = work_model(w, c, wb=wb)
+        A, U, fl, by = work_model(w, c, wb=wb, ab=ab)
         A_steps.append(A)
         U_steps.append(U)
         ffn = c[:w.N]
@@ -264,7 +268,7 @@ def step_work(w, hist, wb=2):
     return tot_flops, tot_bytes, (A_steps, U_steps, load_ratio)
 
 
-def roofline_of(w, stage_ms, tot_flops, tot_bytes, fp8=False):
+def roofline_of(w, stage_ms, tot_flops, tot_bytes, fp8=False, fp8_act=False):
     """Roofline record of the dominant (longest) stage: FLOP/s against the burst bf16 peak for
     a contraction at prefill-like sizes, bytes/s against the HBM copy peak at decode."""
     pk, pk_src = peaks()
@@ -287,7 +291,7 @@ def roofline_of(w, stage_ms, tot_flops, tot_bytes, fp8=False):
     # the datasheet figures (dense bf16 2250 TFLOP/s, HBM3e 8000 GB/s), for context
     roof["frac_of_nominal"] = round(achieved / (NOMINAL_HBM_GBS if roof["bound"] == "hbm"
                                                 else NOMINAL_BF16_TFLOPS), 4)
-    tr = NCU_TRAFFIC.get((w.name + ("+fp8" if fp8 else ""), kernel))
+    tr = NCU_TRAFFIC.get((w.name + ("+fp8" if fp8 else "") + ("+act" if fp8_act else ""), kernel))
     roof["traffic"] = tr["bytes_per_launch"] if tr and tr["src"] == gemm_source_hash() else None
     roof["kernel"] = kernel
     roof["peak_source"] = f"{pk_src} {peak_name}"
@@ -433,7 +437,8 @@ def run_ours(args, rank, world, local_rank):
     wt = make_weights(w, device, seed=args.seed)
     x = make_tokens(w, device, seed=args.seed + rank)
     dm = mb.dims(w.T, w.d, w.N, w.Z, w.K, w.I,
-                 flags=mb.RENORMALIZE_GATES if args.renormalize_gates else 0)
+                 flags=(mb.RENORMALIZE_GATES if args.renormalize_gates else 0) |
+                 (mb.FP8_ACTIVATIONS if args.fp8_activations else 0))
     ws = mb.alloc_workspace(dm, device)
     y = torch.empty((w.T, w.d), dtype=torch.bfloat16, device=device)
     b = wt["b"].clone()
@@ -543,8 +548,10 @@ def run_ours(args, rank, world, local_rank):
     # per-stage durations and algorithmic work of the timed steps
     stage_ms = stage_durations(events)
     hist = counts[args.warmup:n_steps].cpu().numpy()
-    tot_flops, tot_bytes, routing = step_work(w, hist, wb=1 if args.fp8 else 2)
-    roof = roofline_of(w, stage_ms, tot_flops, tot_bytes, fp8=args.fp8)
+    tot_flops, tot_bytes, routing = step_work(w, hist, wb=1 if args.fp8 else 2,
+                                              ab=1 if args.fp8_activations else 2)
+    roof = roofline_of(w, stage_ms, tot_flops, tot_bytes, fp8=args.fp8,
+                       fp8_act=args.fp8_activations)
     layer_flops = sum(tot_flops.values())
     if scmoe is not None:
         scmoe["step_ms"] = round(ms / args.steps, 4)
@@ -633,7 +640,8 @@ def finish(args, w, world, rank, ms_max, routing, roof, layer, stage_ms, clk, e2
         "metric": METRIC, "value": round(job_throughput(world, w.T, args.steps, ms_max), 1),
         "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms_max / args.steps, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3 x e4m3 -> f32" if args.fp8_activations else "bf16",
         "data": "synthetic (seeded; x~N(0,1), weights~N(0,0.02^2) bf16, biases~U(-0.05,0.05))",
         "config": {
             "workload": w.name, "T": w.T, "d": w.d, "N": w.N, "Z": w.Z, "K": w.K, "I": w.I,
@@ -645,6 +653,8 @@ def finish(args, w, world, rank, ms_max, routing, roof, layer, stage_ms, clk, e2
             "variant": {"renormalize_gates": bool(args.renormalize_gates),
                         "balance_gamma": args.balance_gamma,
                         "expert_weights": "fp8 e4m3, 128x128 blocks" if args.fp8 else "bf16",
+                        "activations": "fp8 e4m3, 1x128 blocks (E4M3 x E4M3 MMAs)"
+                                       if args.fp8_activations else "bf16",
                         "scmoe_dense_ffn": args.scmoe or None},
             "mean_ffn_experts_per_token": round(float(np.mean(A_steps)) / w.T, 4),
             "distinct_ffn_experts": int(np.mean(U_steps)),
@@ -656,7 +666,8 @@ def finish(args, w, world, rank, ms_max, routing, roof, layer, stage_ms, clk, e2
         "stages_ms": {k: round(v / args.steps, 4) for k, v in stage_ms.items()},
         "clocks": clk,
         "e2e": e2e,
-        "gpu_launches": (LAUNCHES_PER_STEP + (2 if args.scmoe else 0)) * args.steps,
+        "gpu_launches": (LAUNCHES_PER_STEP + (2 if args.scmoe else 0) +
+                         (1 if args.fp8_activations else 0)) * args.steps,
     }
     if decode is not None:
         result["decode"] = decode
@@ -733,11 +744,16 @@ def main():
                          "shortcut branch) on a second stream beside each step")
     ap.add_argument("--fp8", action="store_true",
                     help="variant: block-wise FP8 (E4M3) expert weights, quantised on the GPU")
+    ap.add_argument("--fp8-activations", action="store_true",
+                    help="variant (with --fp8): E4M3 activations too, 1x128 blocks, read by "
+                         "E4M3 x E4M3 tensor-core MMAs")
     ap.add_argument("--balance-gamma", type=float, default=0.0,
                     help="variant: step of the per-expert balancing term after the PID step")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.fp8_activations and not args.fp8:
+        ap.error("--fp8-activations needs --fp8")
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))

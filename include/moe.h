@@ -53,13 +53,25 @@ typedef struct {
     int32_t Z; /* zero-computation experts (ids N .. N+Z-1) */
     int32_t K; /* experts selected per token */
     int32_t I; /* intermediate width of each SwiGLU FFN expert */
-    uint32_t flags; /* variant switches (MOE_RENORMALIZE_GATES); 0 = the layer as defined */
+    uint32_t flags; /* variant switches (MOE_RENORMALIZE_GATES, MOE_FP8_ACTIVATIONS); 0 = the
+                       layer as defined */
 } moe_dims;
 
 /* Gates renormalised over the selected set: g_i = p_i / sum of p over the K selected experts
  * (zero experts included), instead of the layer's unrenormalised p_i.  An optional variant;
  * it changes moe_route's topk_gate and hence everything downstream, not the selection. */
 #define MOE_RENORMALIZE_GATES 1u
+
+/* FP8 activations, for the FP8-weight entry points only (moe_expert_ffn_fp8, moe_forward_fp8;
+ * the bf16 ones return MOE_ERR_ARG when it is set): the inputs of both expert GEMMs -- the token
+ * rows and h -- are quantised to E4M3 with one power-of-two scale per token per 128 channels
+ * (the activation side of the DeepSeek-V3 block scheme that "衝上熱搜！美團大模型，靠「快」火了",
+ * §系統級優化 names; scale rule and rounding as in moe_quantize_fp8, see moe_quantize_fp8_rows),
+ * and the tensor cores multiply E4M3 by E4M3 with fp32 sums, each 128-long block of the
+ * reduction scaled by its weight and activation scales.  Requires d and I multiples of 128
+ * (MOE_ERR_SHAPE otherwise); the codes and scales of x_perm and h live in the workspace scratch
+ * (moe_scratch_size grows by about T*K*(d + I)*1.03 bytes). */
+#define MOE_FP8_ACTIVATIONS 2u
 
 /* PID gains and set-point: target = desired mean number of FFN experts per token.
  * balance_gamma: step of the per-expert balancing term (see moe_bias_update); 0 = off. */
@@ -272,11 +284,24 @@ int moe_forward_timed(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *W
 int moe_quantize_fp8(const moe_bf16 *w, int64_t G, int64_t R, int64_t C, uint8_t *q,
                      float *scale, void *stream);
 
+/* Block-wise FP8 of activation rows (the MOE_FP8_ACTIVATIONS variant): for each row r of
+ * x [R, C] bf16 and each 1 x 128 block of it, e = the smallest integer with max|x| <= 448 * 2^e
+ * (e >= -126; 0 for an all-zero block) and q = E4M3(x / 2^e), nearest, ties to even (the rule
+ * of moe_quantize_fp8 on 1 x 128 blocks).
+ *   x     [R, C] bf16                C a multiple of 128 (MOE_ERR_SHAPE otherwise)
+ *   q     [R, C] uint8 (out)         E4M3 codes
+ *   scale [C/128, R] fp32 (out)      block-major: scale[(c / 128) * R + r] = 2^e
+ * All pointers 16-byte aligned. */
+int moe_quantize_fp8_rows(const moe_bf16 *x, int64_t R, int64_t C, uint8_t *q, float *scale,
+                          void *stream);
+
 /* moe_expert_ffn with block-quantised expert weights (from moe_quantize_fp8): each weight
  * tile is read as E4M3 codes (half the bytes of bf16) and turned into the exact bf16 weights
  * q * scale in shared memory; activations, accumulation and outputs are as in moe_expert_ffn,
  * so the result equals moe_expert_ffn on the dequantised weights.  d and I must be multiples
- * of 128. */
+ * of 128.  With MOE_FP8_ACTIVATIONS in dims->flags the activations are quantised too and the
+ * tensor cores read E4M3 on both sides (see the flag); h is then unused (may be NULL) and the
+ * quantised h stays in the workspace. */
 int moe_expert_ffn_fp8(const moe_dims *dims, const moe_bf16 *x_perm, const int32_t *offsets,
                        const float *perm_gate, const uint8_t *q_g, const float *s_g,
                        const uint8_t *q_u, const float *s_u, const uint8_t *q_d,

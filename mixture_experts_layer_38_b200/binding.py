@@ -20,7 +20,7 @@ EXPORTS = (
     "moe_expert_ffn", "moe_combine", "moe_bias_update", "moe_forward", "moe_forward_timed",
     "moe_last_device_error", "moe_dispatch_noalloc", "moe_expert_ffn_gather",
     "moe_quantize_fp8", "moe_expert_ffn_fp8", "moe_forward_fp8", "moe_dense_ffn",
-    "moe_router_logits", "moe_debug_set_wait_limit",
+    "moe_router_logits", "moe_debug_set_wait_limit", "moe_quantize_fp8_rows",
 )
 NUM_STAGE_EVENTS = 7
 STAGE_NAMES = ("router_gemm", "route_topk", "dispatch", "ffn_up_gemm", "ffn_down_gemm",
@@ -87,6 +87,7 @@ def lib():
         L.moe_expert_ffn_gather.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]
         _I64 = ctypes.c_int64
         L.moe_quantize_fp8.argtypes = [_P, _I64, _I64, _I64, _P, _P, _P]
+        L.moe_quantize_fp8_rows.argtypes = [_P, _I64, _I64, _P, _P, _P]
         L.moe_dense_ffn.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, _S, _P]
         L.moe_expert_ffn_fp8.argtypes = [_DP] + [_P] * 11 + [_P, _S, _P]
         L.moe_forward_fp8.argtypes = [_DP] + [_P] * 11 + [_P, _S,
@@ -95,13 +96,15 @@ def lib():
                   "moe_bias_update", "moe_forward", "moe_forward_timed",
                   "moe_last_device_error", "moe_dispatch_noalloc", "moe_expert_ffn_gather",
                   "moe_quantize_fp8", "moe_expert_ffn_fp8", "moe_forward_fp8",
-                  "moe_dense_ffn", "moe_router_logits", "moe_debug_set_wait_limit"):
+                  "moe_dense_ffn", "moe_router_logits", "moe_debug_set_wait_limit",
+                  "moe_quantize_fp8_rows"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
 
 
 RENORMALIZE_GATES = 1  # MOE_RENORMALIZE_GATES
+FP8_ACTIVATIONS = 2  # MOE_FP8_ACTIVATIONS
 
 
 def dims(T, d, N, Z, K, I, flags=0) -> Dims:
@@ -321,6 +324,16 @@ def moe_quantize_fp8(w, q, scale, stream=None):
     _check("moe_quantize_fp8", rc)
 
 
+def moe_quantize_fp8_rows(x, q, scale, stream=None):
+    """E4M3 codes of bf16 rows x [R, C] with one power-of-two scale per 1 x 128 block;
+    scale is block-major [C/128, R]."""
+    R, C = x.shape
+    rc = lib().moe_quantize_fp8_rows(
+        _ptr(x, torch.bfloat16, (R, C), "x"), R, C, _ptr(q, torch.uint8, (R, C), "q"),
+        _ptr(scale, torch.float32, (C // 128, R), "scale"), _stream(stream))
+    _check("moe_quantize_fp8_rows", rc)
+
+
 def quantize_expert_weights_fp8(dm, W_g, W_u, W_d, stream=None):
     """All three expert weight tensors quantised on the device: a dict of codes and scales."""
     out = {}
@@ -350,8 +363,8 @@ def moe_expert_ffn_fp8(dm, x_perm, offsets, perm_gate, fw, h, y_perm, ws, stream
         ctypes.byref(dm), _ptr(x_perm, torch.bfloat16, (R, dm.d), "x_perm"),
         _ptr(offsets, torch.int32, (dm.N + 1,), "offsets"),
         _ptr(perm_gate, torch.float32, (R,), "perm_gate"), *_fp8_args(dm, fw),
-        _ptr(h, torch.bfloat16, (R, dm.I), "h"), _ptr(y_perm, torch.bfloat16, (R, dm.d), "y_perm"),
-        w, n, _stream(stream))
+        _ptr(h, torch.bfloat16, (R, dm.I), "h", nullable=bool(dm.flags & FP8_ACTIVATIONS)),
+        _ptr(y_perm, torch.bfloat16, (R, dm.d), "y_perm"), w, n, _stream(stream))
     _check("moe_expert_ffn_fp8", rc)
 
 

@@ -171,6 +171,28 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
 }
 
+// Instruction descriptor of kind::f8f6f4 with E4M3 A and B (both K-major), fp32 accumulator.
+// A K-step of one MMA is 32 elements (32 bytes), like kind::f16's 16 bf16 elements, so the
+// shared-memory descriptors and their per-step advance are the same.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return (1u << 4)                                  // D format: f32
+         | (0u << 7)                                // A format: E4M3
+         | (0u << 10)                               // B format: E4M3
+         | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T with E4M3 operands, one elected thread issues.
+__device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T, one elected thread issues.
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                           uint32_t idesc, uint32_t accumulate) {
@@ -287,6 +309,25 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t *bar, uint16_t cta_mas
       " [%0], %1;" ::"r"(smem_u32(bar)),
       "h"(cta_mask)
       : "memory");
+}
+
+// ---------------------------------------------------------------- FP8 (E4M3) blocks
+// Exponent e of a block's power-of-two scale: the smallest integer with amax <= 448 * 2^e
+// (448 = the largest finite E4M3 value), at least -126; 0 for an all-zero block.
+__device__ __forceinline__ int fp8_scale_exponent(float amax) {
+  if (!(amax > 0.f)) return 0;
+  int x;
+  const float f = frexpf(amax, &x);  // amax = f * 2^x, f in [0.5, 1)
+  const int e = x - 9 + (f > 0.875f ? 1 : 0);  // 448 * 2^e = 0.875 * 2^(e + 9)
+  return e < -126 ? -126 : e;
+}
+
+// 2^e as a float for -126 <= e <= 127 (exact).
+__device__ __forceinline__ float exp2_int(int e) { return __int_as_float((e + 127) << 23); }
+
+// Barrier over the `threads` threads (a multiple of 32) that use barrier `id` (1-15).
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
 // ---------------------------------------------------------------- misc

@@ -53,6 +53,11 @@ struct GemmArgs {
   // Cycles after which one pipeline wait gives up (set by the launchers; see
   // gemm_set_wait_limit).
   long long wait_limit;
+  // E4M3 activations (launch_grouped_gemm_e4m3): the scale of activation row r, columns
+  // [128 kb, 128 kb + 128) is act_scale[kb * rows + r]; with kEpiSwiGLU the kernel writes h as
+  // E4M3 codes (out, [rows, M] bytes) and their scales to out_scale[(f / 128) * rows + r].
+  const float *act_scale;
+  float *out_scale;
 };
 
 // Grouped GEMM block: warp 0 issues TMA loads, warp 1 allocates TMEM and issues MMAs, and
@@ -70,14 +75,22 @@ int gemm_tile_tokens(long long rows, int groups, int K);
 cudaError_t launch_grouped_gemm(int epi, const GemmArgs &args, int grid, int tile_tokens,
                                 cudaStream_t stream);
 // SwiGLU or gated grouped GEMM on CTA pairs (clusters of two SMs, pair MMAs of 256 weight
-// rows) running two pipelines per pair at once: full 192-token tiles (and tails over 64 rows)
-// beside tails of at most 64 rows, so tensor work and weight streaming overlap within each SM.
+// rows) running two pipelines per pair at once: full 224-token tiles (and tails over 32 rows)
+// beside tails of at most 32 rows, so tensor work and weight streaming overlap within each SM.
 // Needs M a multiple of 256 (SwiGLU) or 512 (gated), group row counts within gemm_dual_fits;
 // `pairs` = the persistent pairs to launch (gemm_max_dual_pairs caps it).
 cudaError_t launch_grouped_gemm_dual(int epi, const GemmArgs &args, int pairs,
                                      cudaStream_t stream);
 int gemm_max_dual_pairs(int device);  // co-resident pairs on the device (gemm_prepare queries it)
 bool gemm_dual_fits(long long rows, int groups);
+// SwiGLU or gated grouped GEMM with E4M3 weights AND E4M3 activations (tcgen05.mma
+// kind::f8f6f4): map_a0 / map_a1 cover weight codes and map_b[1..3] activation codes in
+// 128-byte-swizzled boxes of 128 columns (64 / 32 / 16 rows for the tokens); scale_a0/1 and
+// act_scale as described in GemmArgs.  K and M multiples of 128.
+cudaError_t launch_grouped_gemm_e4m3(int epi, const GemmArgs &args, int grid,
+                                     cudaStream_t stream);
+cudaError_t gemm_e4m3_prepare();  // sets the kernels' shared-memory limit (gemm_prepare calls it)
+long long gemm_wait_limit();      // the current gemm_set_wait_limit value (0: the default)
 // SwiGLU or gated grouped GEMM with E4M3 block-quantised weights, 128-token tiles.
 cudaError_t launch_grouped_gemm_fp8(int epi, const GemmArgs &args, int grid,
                                     cudaStream_t stream);
@@ -86,6 +99,12 @@ cudaError_t launch_grouped_gemm_fp8(int epi, const GemmArgs &args, int grid,
 // scale per 128 x 128 block.
 cudaError_t launch_quantize_fp8(const uint16_t *w, long long G, long long R, long long C,
                                 uint8_t *q, float *scale, cudaStream_t stream);
+
+// FP8 activations: rows of the bf16 matrix x [R, C] (C a multiple of 128) -> E4M3 codes q
+// [R, C] and one power-of-two scale per 1 x 128 block, stored block-major:
+// scale_t[(c / 128) * R + r].  Rows from *live_rows on are skipped (live_rows may be NULL).
+cudaError_t launch_quantize_fp8_rows(const uint16_t *x, long long R, int C, const int *live_rows,
+                                     uint8_t *q, float *scale_t, cudaStream_t stream);
 
 // ------------------------------------------------------------------ routing
 // logits [splits][T][E] fp32 -> softmax, biased top-K, ascending ids.

@@ -109,6 +109,22 @@ bool make_map_u8(CUtensorMap *map, const void *base, uint64_t rows, uint64_t col
          CUDA_SUCCESS;
 }
 
+// Row-major E4M3 codes [rows, cols] in boxes of 128 columns (128 bytes) x box_rows rows with the
+// 128-byte swizzle: the operand layout the kind::f8f6f4 MMAs read (FP8 activations).
+bool make_map_e4m3(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                   uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estride[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box,
+            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 // Block-quantised expert weights: E4M3 codes in the bf16 weights' layouts and one fp32
 // power-of-two scale per 128 x 128 block ([N][rows / 128][cols / 128]).
 struct Fp8Weights {
@@ -150,12 +166,16 @@ bool dims_ok(const moe_dims *d) {
   if (d->K < 1 || d->K > kMaxK || d->K > E) return false;
   if ((long long)d->T * d->K >= (1ll << 31)) return false;
   if ((long long)d->N * d->I >= (1ll << 31) || (long long)d->N * d->d >= (1ll << 31)) return false;
-  if ((d->flags & ~MOE_RENORMALIZE_GATES) != 0) return false;
+  if ((d->flags & ~(MOE_RENORMALIZE_GATES | MOE_FP8_ACTIVATIONS)) != 0) return false;
+  // FP8 activations are scaled per 128 channels (and need FP8 weights, whose blocks are 128).
+  if ((d->flags & MOE_FP8_ACTIVATIONS) && (d->d % 128 != 0 || d->I % 128 != 0)) return false;
   return true;
 }
 
 // The FP8 weight path scales 128 x 128 blocks: both GEMMs' dims must be whole blocks.
 bool fp8_dims_ok(const moe_dims &d) { return d.d % 128 == 0 && d.I % 128 == 0; }
+
+bool fp8_act(const moe_dims &d) { return (d.flags & MOE_FP8_ACTIVATIONS) != 0; }
 
 int router_splits(const moe_dims &d) {
   const int E = d.N + d.Z;
@@ -171,7 +191,7 @@ int router_splits(const moe_dims &d) {
 struct Layout {
   int splits;
   int epad;
-  size_t status, logits, chunk, scratch_end;
+  size_t status, logits, chunk, xq, sx, hq, sh, scratch_end;
   size_t topk_idx, topk_gate, gap, counts, offsets, perm_tok, perm_gate, slot_pos;
   size_t x_perm, h, y_perm, total;
 };
@@ -191,6 +211,12 @@ Layout layout_of(const moe_dims &d) {
   L.status = take(kAlign);
   L.logits = take((size_t)L.splits * T * L.epad * 4);
   L.chunk = take((size_t)dispatch_chunks(d.T) * E * 4);
+  if (d.flags & MOE_FP8_ACTIVATIONS) {  // E4M3 codes and block scales of x_perm and h
+    L.xq = take(rows * (size_t)d.d);
+    L.sx = take(rows * (size_t)(d.d / 128) * 4);
+    L.hq = take(rows * (size_t)d.I);
+    L.sh = take(rows * (size_t)(d.I / 128) * 4);
+  }
   L.scratch_end = off;
   L.topk_idx = take(rows * 4);
   L.topk_gate = take(rows * 4);
@@ -392,6 +418,70 @@ int do_expert_ffn(const moe_dims &d, const DeviceInfo &di, const Layout &L,
   return to_status(launch_grouped_gemm(kEpiGated, down, di.sms, tile_tokens, stream));
 }
 
+// The expert FFN with FP8 weights and FP8 activations: x_perm's rows are quantised (1 x 128
+// blocks) into the workspace, the up-projection reads the codes on the tensor cores and writes
+// h as codes and scales, and the down projection reads those.
+int do_expert_ffn_e4m3(const moe_dims &d, const DeviceInfo &di, const Layout &L,
+                       const moe_bf16 *x_perm, const int32_t *offsets, const float *perm_gate,
+                       const Fp8Weights &fw, moe_bf16 *y_perm, void *ws, cudaStream_t stream,
+                       void *const *events = nullptr) {
+  if (d.T == 0 || d.N == 0) return record(events, 4, stream);
+  const uint64_t rows = (uint64_t)d.T * d.K;
+  int *status = at<int>(ws, L.status);
+  uint8_t *xq = at<uint8_t>(ws, L.xq);
+  float *sx = at<float>(ws, L.sx);
+  uint8_t *hq = at<uint8_t>(ws, L.hq);
+  float *sh = at<float>(ws, L.sh);
+  // Only the rows of the FFN experts' groups (offsets[N] of them) are quantised.
+  if (launch_quantize_fp8_rows(x_perm, (long long)rows, d.d, offsets + d.N, xq, sx, stream) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  GemmArgs up{};
+  bool ok = make_map_e4m3(&up.map_a0, fw.q_g, (uint64_t)d.N * d.I, (uint64_t)d.d, 128) &&
+            make_map_e4m3(&up.map_a1, fw.q_u, (uint64_t)d.N * d.I, (uint64_t)d.d, 128);
+  for (int i = 1; i < 4 && ok; ++i)
+    ok = make_map_e4m3(&up.map_b[i], xq, rows, (uint64_t)d.d, 128u >> i);
+  if (!ok) return MOE_ERR_CUDA;
+  up.group_offsets = offsets;
+  up.num_groups = d.N;
+  up.rows = (int)rows;
+  up.M = d.I;
+  up.K = d.d;
+  up.k_splits = 1;
+  up.out = hq;
+  up.out_ld = d.I;
+  up.status = status;
+  up.scale_a0 = fw.s_g;
+  up.scale_a1 = fw.s_u;
+  up.scale_ld = d.d / 128;
+  up.act_scale = sx;
+  up.out_scale = sh;
+  if (launch_grouped_gemm_e4m3(kEpiSwiGLU, up, di.sms, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  if (record(events, 4, stream) != MOE_OK) return MOE_ERR_CUDA;
+
+  GemmArgs down{};
+  ok = make_map_e4m3(&down.map_a0, fw.q_d, (uint64_t)d.N * d.d, (uint64_t)d.I, 128) &&
+       make_map_e4m3(&down.map_a1, fw.q_d, (uint64_t)d.N * d.d, (uint64_t)d.I, 128);
+  for (int i = 1; i < 4 && ok; ++i)
+    ok = make_map_e4m3(&down.map_b[i], hq, rows, (uint64_t)d.I, 128u >> i);
+  if (!ok) return MOE_ERR_CUDA;
+  down.group_offsets = offsets;
+  down.num_groups = d.N;
+  down.rows = (int)rows;
+  down.M = d.d;
+  down.K = d.I;
+  down.k_splits = 1;
+  down.out = y_perm;
+  down.out_ld = d.d;
+  down.row_scale = perm_gate;
+  down.status = status;
+  down.scale_a0 = fw.s_d;
+  down.scale_a1 = fw.s_d;
+  down.scale_ld = d.I / 128;
+  down.act_scale = sh;
+  return to_status(launch_grouped_gemm_e4m3(kEpiGated, down, di.sms, stream));
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -475,6 +565,7 @@ int moe_expert_ffn(const moe_dims *dims, const moe_bf16 *x_perm, const int32_t *
                    size_t ws_bytes, void *stream) {
   MOE_REQUIRE(dims != nullptr, MOE_ERR_ARG);
   MOE_REQUIRE(dims_ok(dims), MOE_ERR_SHAPE);
+  MOE_REQUIRE(!fp8_act(*dims), MOE_ERR_ARG);  // FP8 activations need FP8 weights
   MOE_CHECK_TOKEN_PTR(x_perm, dims->T);
   MOE_CHECK_PTR(offsets);
   MOE_CHECK_TOKEN_PTR(perm_gate, dims->T);
@@ -499,6 +590,7 @@ int moe_expert_ffn_gather(const moe_dims *dims, const moe_bf16 *x, const int32_t
                           moe_bf16 *y_perm, void *ws, size_t ws_bytes, void *stream) {
   MOE_REQUIRE(dims != nullptr, MOE_ERR_ARG);
   MOE_REQUIRE(dims_ok(dims), MOE_ERR_SHAPE);
+  MOE_REQUIRE(!fp8_act(*dims), MOE_ERR_ARG);
   MOE_CHECK_TOKEN_PTR(x, dims->T);
   MOE_CHECK_TOKEN_PTR(perm_tok, dims->T);
   MOE_CHECK_PTR(offsets);
@@ -656,6 +748,7 @@ int forward_impl(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *W_r, c
   MOE_CHECK_PTR(W_r);
   MOE_CHECK_PTR(b);
   if (fw == nullptr) {
+    MOE_REQUIRE(!fp8_act(*dims), MOE_ERR_ARG);  // FP8 activations need FP8 weights
     MOE_CHECK_PTR(W_g);
     MOE_CHECK_PTR(W_u);
     MOE_CHECK_PTR(W_d);
@@ -700,8 +793,10 @@ int forward_impl(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *W_r, c
                    slot_pos, x_perm, ws, s);
   if (rc != MOE_OK) return rc;
   if ((rc = record(ev, 3, s)) != MOE_OK) return rc;
-  rc = do_expert_ffn(d, *di, L, x_perm, offsets, perm_gate, W_g, W_u, W_d, h, y_perm, ws, s, ev,
-                     nullptr, nullptr, fw);
+  rc = fw != nullptr && fp8_act(d)
+           ? do_expert_ffn_e4m3(d, *di, L, x_perm, offsets, perm_gate, *fw, y_perm, ws, s, ev)
+           : do_expert_ffn(d, *di, L, x_perm, offsets, perm_gate, W_g, W_u, W_d, h, y_perm, ws,
+                           s, ev, nullptr, nullptr, fw);
   if (rc != MOE_OK) return rc;
   if ((rc = record(ev, 5, s)) != MOE_OK) return rc;
   rc = to_status(launch_combine(x, y_perm, topk_idx, topk_gate, slot_pos, d.T, d.d, d.N, d.K,
@@ -747,6 +842,21 @@ int moe_quantize_fp8(const moe_bf16 *w, int64_t G, int64_t R, int64_t C, uint8_t
   return to_status(launch_quantize_fp8(w, G, R, C, q, scale, static_cast<cudaStream_t>(stream)));
 }
 
+int moe_quantize_fp8_rows(const moe_bf16 *x, int64_t R, int64_t C, uint8_t *q, float *scale,
+                          void *stream) {
+  MOE_REQUIRE(R >= 0 && C >= 0 && C % 128 == 0 && C < (1ll << 31), MOE_ERR_SHAPE);
+  MOE_REQUIRE(R <= ((1ll << 31) - 1) * 8 / std::max<int64_t>(1, (C / 128 + 1) / 2), MOE_ERR_SHAPE);
+  if (R == 0 || C == 0) return MOE_OK;
+  MOE_CHECK_PTR(x);
+  MOE_CHECK_PTR(q);
+  MOE_CHECK_PTR(scale);
+  const DeviceInfo *di = nullptr;
+  const int rc = device_info(&di);
+  if (rc != MOE_OK) return rc;
+  return to_status(launch_quantize_fp8_rows(x, R, (int)C, nullptr, q, scale,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
 int moe_expert_ffn_fp8(const moe_dims *dims, const moe_bf16 *x_perm, const int32_t *offsets,
                        const float *perm_gate, const uint8_t *q_g, const float *s_g,
                        const uint8_t *q_u, const float *s_u, const uint8_t *q_d,
@@ -764,7 +874,7 @@ int moe_expert_ffn_fp8(const moe_dims *dims, const moe_bf16 *x_perm, const int32
   MOE_CHECK_PTR(s_g);
   MOE_CHECK_PTR(s_u);
   MOE_CHECK_PTR(s_d);
-  MOE_CHECK_TOKEN_PTR(h, dims->T);
+  if (!fp8_act(*dims)) MOE_CHECK_TOKEN_PTR(h, dims->T);  // unused with FP8 activations
   MOE_CHECK_TOKEN_PTR(y_perm, dims->T);
   const Layout L = layout_of(*dims);
   int rc = check_ws(ws, ws_bytes, L.scratch_end);
@@ -772,6 +882,9 @@ int moe_expert_ffn_fp8(const moe_dims *dims, const moe_bf16 *x_perm, const int32
   const DeviceInfo *di = nullptr;
   rc = device_info(&di);
   if (rc != MOE_OK) return rc;
+  if (fp8_act(*dims))
+    return do_expert_ffn_e4m3(*dims, *di, L, x_perm, offsets, perm_gate, fw, y_perm, ws,
+                              static_cast<cudaStream_t>(stream));
   return do_expert_ffn(*dims, *di, L, x_perm, offsets, perm_gate, nullptr, nullptr, nullptr, h,
                        y_perm, ws, static_cast<cudaStream_t>(stream), nullptr, nullptr, nullptr,
                        &fw);

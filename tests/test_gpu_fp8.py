@@ -6,6 +6,13 @@
   * moe_expert_ffn_fp8 / moe_forward_fp8: within the output tolerances of the oracle run on
     the dequantised weights, and bit-identical to the bf16 path given those same dequantised
     weights (the E4M3 -> bf16 step is exact, the tensor-core path is shared).
+FP8 activations (MOE_FP8_ACTIVATIONS: E4M3 x E4M3 on the tensor cores):
+  * moe_quantize_fp8_rows: codes and block scales bit-exact with the oracle's 1 x 128 row
+    quantisation, special blocks included;
+  * moe_expert_ffn_fp8 / moe_forward_fp8 with the flag: within the output tolerances of the
+    oracle's FP8-activation expert on the dequantised weights, over several token tiles per
+    expert and ragged tails; and measurably different from the bf16-activation result, so the
+    comparison sees the quantisation.
 Page cited: "衝上熱搜！美團大模型，靠「快」火了", section 系統級優化 (block-wise quantisation as in
 DeepSeek-V3).
 """
@@ -119,3 +126,94 @@ def test_forward_fp8_tiny_matches_oracle():
                    wt_deq["W_u"].to(DEV), wt_deq["W_d"].to(DEV), y2, None, ws)
     torch.cuda.synchronize()
     assert torch.equal(y, y2)
+
+
+# ------------------------------------------------------------------ FP8 activations
+
+def _special_rows(R, C, seed):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn((R, C), generator=g)
+    x[0, :128] = 0                                        # an all-zero block
+    if C >= 256:
+        x[1, 128:256] *= 3000                             # a wide-range block
+        x[2, 128:256] *= 1e-30                            # tiny values (scale near 2^-126)
+    # exact rounding ties after scaling: amax 3 (e = -7), (1 + 1/16) * 2^k halfway between codes
+    x[3, :128] = 0
+    x[3, 0] = 3.0
+    for i, k in enumerate(range(-16, -6)):
+        x[3, 1 + i] = (1 + 1 / 16) * 2.0 ** k
+        x[3, 20 + i] = -(1 + 3 / 16) * 2.0 ** k
+    x[4, :] = -0.0
+    return x.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("R,C", [(5, 128), (37, 384), (1139, 6144)])
+def test_quantize_rows_bit_exact_with_oracle(R, C):
+    x = _special_rows(R, C, seed=R + C)
+    q = torch.empty((R, C), dtype=torch.uint8, device=DEV)
+    s = torch.empty((C // 128, R), dtype=torch.float32, device=DEV)
+    mb.moe_quantize_fp8_rows(x.to(DEV), q, s)
+    torch.cuda.synchronize()
+    q_ref, s_ref = oracle.quantize_fp8_rows(x.double().numpy())
+    np.testing.assert_array_equal(s.cpu().numpy().T, s_ref)
+    np.testing.assert_array_equal(q.cpu().numpy(), q_ref)
+
+
+def _fp8act_rows(w, st, x, wt_deq, A):
+    xb = oracle.bf16_bits(x)
+    perm, offs, gates = to_np(st.perm_tok)[:A], to_np(st.offsets), to_np(st.perm_gate)[:A]
+    rows = np.zeros((A, w.d))
+    for e in range(w.N):
+        lo, hi = offs[e], offs[e + 1]
+        if hi > lo:
+            rows[lo:hi] = gates[lo:hi, None].astype(np.float64) * oracle.swiglu_expert(
+                xb[perm[lo:hi]], wt_deq["W_g"][e], wt_deq["W_u"][e], wt_deq["W_d"][e],
+                fp8_act=True)
+    return rows
+
+
+def _rel_l2(a, b):
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+# 64-token tiles: several per expert and ragged tails at mid T = 1500 (9000 rows, 64 experts),
+# one partial tile per expert at T = 333 and tiny
+@pytest.mark.parametrize("name,T", [("tiny", None), ("mid", 333), ("mid", 1500)])
+def test_expert_ffn_fp8_activations_match_oracle(name, T):
+    w, x, wt, fw, wt_deq = _fp8_case(name, T)
+    st = Stages(w, x, wt_deq)
+    st.route()
+    st.dispatch()
+    A = int(st.offsets[-1].item())
+    mb.moe_expert_ffn_fp8(st.dm, st.x_perm, st.offsets, st.perm_gate, fw, st.h, st.y_perm,
+                          st.ws)  # bf16 activations, for the contrast below
+    torch.cuda.synchronize()
+    y_bf16act = oracle.bf16_to_f64(to_np(st.y_perm)[:A])
+    dm = mb.dims(w.T, w.d, w.N, w.Z, w.K, w.I, flags=mb.FP8_ACTIVATIONS)
+    ws = mb.alloc_workspace(dm, DEV, scratch_only=True)
+    y_perm = torch.zeros_like(st.y_perm)
+    mb.moe_expert_ffn_fp8(dm, st.x_perm, st.offsets, st.perm_gate, fw, None, y_perm, ws)
+    torch.cuda.synchronize()
+    assert mb.moe_last_device_error(ws) == 0
+    got = oracle.bf16_to_f64(to_np(y_perm)[:A])
+    ref = _fp8act_rows(w, st, x, wt_deq, A)
+    assert_y_close(got, ref, f"{name} fp8-activation y_perm")
+    # the activation quantisation is visible: the bf16-activation rows differ from the
+    # reference far more than the tolerance the FP8-activation rows meet
+    assert _rel_l2(y_bf16act, ref) > 10 * max(_rel_l2(got, ref), 1e-4)
+
+
+def test_forward_fp8_activations_tiny_matches_oracle():
+    w, x, wt, fw, wt_deq = _fp8_case("tiny", seed=5)
+    dm = mb.dims(w.T, w.d, w.N, w.Z, w.K, w.I, flags=mb.FP8_ACTIVATIONS)
+    ws = mb.alloc_workspace(dm, DEV)
+    y = torch.zeros((w.T, w.d), dtype=torch.bfloat16, device=DEV)
+    counts = torch.zeros(w.E, dtype=torch.int32, device=DEV)
+    mb.moe_forward_fp8(dm, x.to(DEV), wt["W_r"].to(DEV), wt["b"].to(DEV), fw, y, counts, ws)
+    torch.cuda.synchronize()
+    assert mb.moe_last_device_error(ws) == 0
+    r = oracle.router(x, wt["W_r"], wt["b"], w.K)
+    ref = oracle.combine_tokens(np.arange(w.T), x, r["topk_idx"], r["topk_gate"], wt_deq["W_g"],
+                                wt_deq["W_u"], wt_deq["W_d"], w.N, fp8_act=True)
+    assert int(counts.sum().item()) == w.T * w.K
+    assert_y_close(oracle.bf16_to_f64(to_np(y)), ref, "tiny fp8-activation forward")

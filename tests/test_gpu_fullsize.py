@@ -188,4 +188,18 @@ def test_decode_fp8_full_size(big_weights):
                                  routing=gpu_routing_for_oracle(idx, ref, tokens))
     y_s = oracle.bf16_to_f64(to_np(y))[tokens]
     assert_y_close(y_s, out["y"], "decode fp8 y")
-    del fw
+
+    # FP8 activations too (the benchmark's --fp8 --fp8-activations leg): the same routing, the
+    # oracle's FP8-activation experts on the same sampled tokens
+    dm8 = mb.dims(w.T, w.d, w.N, w.Z, w.K, w.I, flags=mb.FP8_ACTIVATIONS)
+    ws8 = mb.alloc_workspace(dm8, DEV)
+    y8 = torch.empty_like(y)
+    mb.moe_forward_fp8(dm8, x, big_weights["W_r"], big_weights["b"], fw, y8, None, ws8)
+    torch.cuda.synchronize()
+    assert mb.moe_last_device_error(ws8) == 0
+    out8 = oracle.forward_sampled(np.arange(len(tokens)), oracle.bf16_bits(x.cpu())[tokens], W_r,
+                                  b, w.N, w.Z, w.K, fetch_deq,
+                                  routing=gpu_routing_for_oracle(idx, ref, tokens), fp8_act=True)
+    y8_s = oracle.bf16_to_f64(to_np(y8))[tokens]
+    assert_y_close(y8_s, out8["y"], "decode fp8-activation y")
+    del ws8, fw

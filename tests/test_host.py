@@ -127,6 +127,40 @@ def test_fp8_shape_errors_before_device_work():
                                mb.workspace_size(dm2), None, None) == 1
 
 
+def test_fp8_activation_flag_layout_and_errors():
+    lib = mb.lib()
+    T, d, N, Z, K, I = 64, 256, 8, 4, 3, 384
+    plain = mb.dims(T, d, N, Z, K, I)
+    dm = mb.dims(T, d, N, Z, K, I, flags=mb.FP8_ACTIVATIONS)
+    # the scratch grows by the codes and block scales of x_perm and h (256-byte aligned regions)
+    rows = T * K
+    extra = sum(-(-b // 256) * 256 for b in (rows * d, rows * d // 128 * 4, rows * I,
+                                             rows * I // 128 * 4))
+    assert mb.scratch_size(dm) == mb.scratch_size(plain) + extra
+    assert mb.workspace_size(dm) == mb.workspace_size(plain) + extra
+    # widths that are not whole 128-channel blocks are rejected with the flag only
+    assert mb.workspace_size(mb.dims(T, 192, N, Z, K, I)) > 0
+    assert mb.workspace_size(mb.dims(T, 192, N, Z, K, I, flags=mb.FP8_ACTIVATIONS)) == 0
+    assert mb.workspace_size(mb.dims(T, d, N, Z, K, 320, flags=mb.FP8_ACTIVATIONS)) == 0
+    # the bf16 entry points refuse the flag (MOE_ERR_ARG), before any device work
+    assert _fwd(dm) == 1
+    assert lib.moe_expert_ffn(ctypes.byref(dm), *[P(0x10000 * (i + 1)) for i in range(8)],
+                              P(0x1000000), mb.scratch_size(dm), None) == 1
+    # the FP8 stage call takes h = NULL with the flag, and needs the larger scratch
+    args = [P(0x10000 * (i + 1)) for i in range(9)]  # x_perm, offsets, perm_gate, 6 FP8 tensors
+    assert lib.moe_expert_ffn_fp8(ctypes.byref(dm), *args, None, P(0x200000), P(0x1000000),
+                                  mb.scratch_size(dm) - 256, None) == 4
+    assert lib.moe_expert_ffn_fp8(ctypes.byref(plain), *args, None, P(0x200000), P(0x1000000),
+                                  mb.scratch_size(plain), None) == 1  # h required without it
+    # the row quantiser's shape checks
+    assert lib.moe_quantize_fp8_rows(P(0x10000), 4, 192, P(0x20000), P(0x30000), None) == 2
+    assert lib.moe_quantize_fp8_rows(P(0x10000), -1, 128, P(0x20000), P(0x30000), None) == 2
+    assert lib.moe_quantize_fp8_rows(None, 0, 128, None, None, None) == 0  # nothing to do
+    assert lib.moe_quantize_fp8_rows(P(0x10000), 1 << 40, 1 << 20, P(0x20000), P(0x30000),
+                                     None) == 2  # too many warps for one grid
+    assert lib.moe_quantize_fp8_rows(P(0x10008), 4, 128, P(0x20000), P(0x30000), None) == 3
+
+
 def test_dense_ffn_argument_errors():
     lib = mb.lib()
     for bad in [(64, 100, 1, 0, 1, 256), (64, 128, 1, 0, 1, 96), (-1, 128, 1, 0, 1, 256)]:
@@ -144,7 +178,7 @@ def test_variant_switches_are_validated():
     lib = mb.lib()
     dm = mb.dims(64, 128, 8, 4, 3, 256, flags=mb.RENORMALIZE_GATES)
     assert mb.workspace_size(dm) == mb.workspace_size(mb.dims(64, 128, 8, 4, 3, 256))
-    assert mb.workspace_size(mb.dims(64, 128, 8, 4, 3, 256, flags=2)) == 0  # unknown flag
+    assert mb.workspace_size(mb.dims(64, 128, 8, 4, 3, 256, flags=4)) == 0  # unknown flag
     assert _fwd(mb.dims(64, 128, 8, 4, 3, 256, flags=0x80)) == 2            # MOE_ERR_SHAPE
     for gamma in (float("nan"), float("inf")):
         params = mb.PidParams(8.0, 0.1, 0.0, 0.0, gamma)
