@@ -27,9 +27,11 @@
 //               codes are rounded once from fp32 and stored as [rows, I] bytes.
 //   kEpiGated   y_perm = gate * (down-projection), bf16, as the bf16 kernel's gated epilogue.
 //
-// Warp roles (192 threads, one CTA per SM, persistent): warp 0 TMA producer, warp 1 TMEM
+// Warp roles (224 threads, one CTA per SM, persistent): warp 0 TMA producer, warp 1 TMEM
 // allocator and MMA issuer, warps 2-5 promotion and epilogue (warp w reads TMEM lane quarter
-// w mod 4).  Every wait is bounded; on timeout the kernel records MOE_DEV_WAIT_TIMEOUT and all
+// w mod 4), warp 6 loads each block's scales (s_x per token times s_w per sub-tile) into a
+// shared-memory slot per partial-sum buffer, up to four blocks ahead of the promotion, so the
+// promotion never waits on a global load.  Every wait is bounded; on timeout the kernel records MOE_DEV_WAIT_TIMEOUT and all
 // roles unwind (the epilogue warps agree on stopping before their shared barriers, so none is
 // left waiting at one), in-flight copies and MMAs are drained and TMEM is freed.
 #include <cuda_fp8.h>
@@ -49,15 +51,18 @@ constexpr int kF8Stages = 5;
 constexpr int kF8Parts = 4;                           // TMEM partial-sum buffers
 constexpr int kF8PartCols = 2 * kF8BN;                // sub-tile 0 | sub-tile 1
 constexpr int kF8EpiWarps = 4;
-constexpr int kF8Threads = 64 + 32 * kF8EpiWarps;
+constexpr int kF8ScaleWarp = 2 + kF8EpiWarps;         // warp 6: block-scale loader
+constexpr int kF8Threads = 32 * (kF8ScaleWarp + 1);
 constexpr int kF8StageBytes = 2048;                   // per epilogue warp: output staging
-constexpr int kF8ScaleBytes = 4 * kF8BN * 4;          // per epilogue warp: 2 x 64 block scales
-constexpr int kF8EpiBytes = kF8StageBytes + kF8ScaleBytes;
+constexpr int kF8GateBytes = kF8BN * 4;               // per epilogue warp: the tile's gates
+constexpr int kF8EpiBytes = kF8StageBytes + kF8GateBytes;
+constexpr int kF8SlotFloats = 2 * kF8BN;              // per partial sum: s_x * s_w0, s_x * s_w1
+constexpr int kF8ScaleRing = kF8Parts * kF8SlotFloats * 4;
 constexpr int kF8Shared = 4 * kF8BN * 4 + kF8BN * 4 + 16;  // column maxima, exponents, stop flag
 constexpr int kF8Prefix = 2 * (kMaxGroups + 4) * 4;
-constexpr int kF8NumBars = 2 * kF8Stages + 2 * kF8Parts + 1;
-constexpr int kF8Smem = 1024 + kF8Stages * kF8Stage + kF8EpiWarps * kF8EpiBytes + kF8Shared +
-                        kF8Prefix + kF8NumBars * 8 + 16;
+constexpr int kF8NumBars = 2 * kF8Stages + 4 * kF8Parts + 1;
+constexpr int kF8Smem = 1024 + kF8Stages * kF8Stage + kF8EpiWarps * kF8EpiBytes + kF8ScaleRing +
+                        kF8Shared + kF8Prefix + kF8NumBars * 8 + 16;
 static_assert(kF8Parts * kF8PartCols <= kTmemCols, "TMEM holds 512 columns");
 static_assert(kF8Smem <= 232448, "shared memory per block");
 static_assert(kF8Stage % 1024 == 0 && kF8TileA % 1024 == 0, "1024-byte-aligned operand tiles");
@@ -96,17 +101,21 @@ __global__ void __launch_bounds__(kF8Threads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t *ring = smem;
   uint8_t *epi = smem + kF8Stages * kF8Stage;
-  float *colmax = reinterpret_cast<float *>(epi + kF8EpiWarps * kF8EpiBytes);  // [4][64]
+  float *scale_ring = reinterpret_cast<float *>(epi + kF8EpiWarps * kF8EpiBytes);
+  float *colmax = scale_ring + kF8Parts * kF8SlotFloats;                        // [4][64]
   int *bexp = reinterpret_cast<int *>(colmax + 4 * kF8BN);                     // [64]
   volatile int *stop_flag = reinterpret_cast<volatile int *>(bexp + kF8BN);
-  int *hpre = reinterpret_cast<int *>(epi + kF8EpiWarps * kF8EpiBytes + kF8Shared);
+  int *hpre = reinterpret_cast<int *>(epi + kF8EpiWarps * kF8EpiBytes + kF8ScaleRing +
+                                     kF8Shared);
   int *lpre = hpre + kMaxGroups + 4;
   uint64_t *bars = reinterpret_cast<uint64_t *>(hpre + 2 * (kMaxGroups + 4));
   uint64_t *full_bar = bars;
   uint64_t *empty_bar = bars + kF8Stages;
   uint64_t *pfull_bar = bars + 2 * kF8Stages;
   uint64_t *pempty_bar = pfull_bar + kF8Parts;
-  uint64_t *drain_bar = pempty_bar + kF8Parts;
+  uint64_t *sfull_bar = pempty_bar + kF8Parts;   // the slot's block scales are written
+  uint64_t *sempty_bar = sfull_bar + kF8Parts;   // the epilogue has used them
+  uint64_t *drain_bar = sempty_bar + kF8Parts;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kF8NumBars);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -123,6 +132,8 @@ __global__ void __launch_bounds__(kF8Threads, 1)
     for (int b = 0; b < kF8Parts; ++b) {
       mbar_init(&pfull_bar[b], 1);
       mbar_init(&pempty_bar[b], kF8EpiWarps);
+      mbar_init(&sfull_bar[b], 1);
+      mbar_init(&sempty_bar[b], kF8EpiWarps);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -247,19 +258,47 @@ __global__ void __launch_bounds__(kF8Threads, 1)
         while (!mbar_try_wait(drain_bar, 0) && clock64() - t0 < kDrainLimitCycles) {}
       }
     }
+  } else if (warp == kF8ScaleWarp) {
+    // ---------------------------------------------------------------- block-scale loader
+    long long n = 0;
+    bool ok = true;
+    for (int tile = unit; ok && tile < sched.total; tile += units) {
+      const Tile t = decode_tile<EPI, kF8BN>(args, sched, tile);
+      const float *ws0 = args.scale_a0 + (long long)(t.a0_row / 128) * args.scale_ld;
+      const float *ws1 = args.scale_a1 + (long long)(t.a1_row / 128) * args.scale_ld;
+      for (int kb = 0; kb < KB; ++kb, ++n) {
+        const float sw0 = __ldg(ws0 + kb);
+        const float sw1 = t.has_a1 ? __ldg(ws1 + kb) : 0.f;
+        const float *sx = args.act_scale + (long long)kb * args.rows + t.row0;
+        const float x0 = lane < t.n_valid ? __ldg(sx + lane) : 0.f;
+        const float x1 = lane + 32 < t.n_valid ? __ldg(sx + lane + 32) : 0.f;
+        const int pb = (int)(n % kF8Parts);
+        const uint32_t use = (uint32_t)(n / kF8Parts);
+        if (!warp_wait(&sempty_bar[pb], (use & 1) ^ 1, abort_flag, wlim)) {
+          if (lane == 0) signal_abort(args, abort_flag);
+          ok = false;
+          break;
+        }
+        float *slot = scale_ring + pb * kF8SlotFloats;
+        slot[lane] = x0 * sw0;
+        slot[32 + lane] = x1 * sw0;
+        slot[64 + lane] = x0 * sw1;
+        slot[96 + lane] = x1 * sw1;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sfull_bar[pb]);
+      }
+    }
   } else {
     // ---------------------------------------------------------------- promotion + epilogue
     const int q = warp & 3;
     const int ew = warp - 2;
     uint8_t *stage_bytes = epi + ew * kF8EpiBytes;
-    float *sc = reinterpret_cast<float *>(stage_bytes + kF8StageBytes);  // [2][64]
+    float *gates = reinterpret_cast<float *>(stage_bytes + kF8StageBytes);  // [64]
     long long n = 0;
     bool ok = true;
     for (int tile = unit; tile < sched.total; tile += units) {
       const Tile t = decode_tile<EPI, kF8BN>(args, sched, tile);
       const int chunks = (t.nb + 31) / 32;
-      const float *ws0 = args.scale_a0 + (long long)(t.a0_row / 128) * args.scale_ld;
-      const float *ws1 = args.scale_a1 + (long long)(t.a1_row / 128) * args.scale_ld;
       float acc0[kF8BN], acc1[kF8BN];
 #pragma unroll
       for (int j = 0; j < kF8BN; ++j) {
@@ -267,25 +306,17 @@ __global__ void __launch_bounds__(kF8Threads, 1)
         acc1[j] = 0.f;
       }
       for (int kb = 0; kb < KB; ++kb, ++n) {
-        // This block's scales: s_x(token) * s_w(sub-tile), tokens past the tile's rows 0.
-        const float sw0 = __ldg(ws0 + kb);
-        const float sw1 = t.has_a1 ? __ldg(ws1 + kb) : 0.f;
-        const float *sx = args.act_scale + (long long)kb * args.rows + t.row0;
-        const float x0 = lane < t.n_valid ? __ldg(sx + lane) : 0.f;
-        const float x1 = lane + 32 < t.n_valid ? __ldg(sx + lane + 32) : 0.f;
-        sc[lane] = x0 * sw0;
-        sc[32 + lane] = x1 * sw0;
-        sc[64 + lane] = x0 * sw1;
-        sc[96 + lane] = x1 * sw1;
-        __syncwarp();
         const int pb = (int)(n % kF8Parts);
         const uint32_t use = (uint32_t)(n / kF8Parts);
-        if (!warp_wait(&pfull_bar[pb], use & 1, abort_flag, wlim)) {
+        // This block's scales s_x(token) * s_w(sub-tile) (0 past the tile's rows), then the sums.
+        if (!warp_wait(&sfull_bar[pb], use & 1, abort_flag, wlim) ||
+            !warp_wait(&pfull_bar[pb], use & 1, abort_flag, wlim)) {
           if (lane == 0) signal_abort(args, abort_flag);
           ok = false;
           break;
         }
         tc_fence_after();
+        const float *sc = scale_ring + pb * kF8SlotFloats;
         const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + pb * kF8PartCols;
 #pragma unroll
         for (int c = 0; c < kF8BN / 32; ++c) {
@@ -316,6 +347,7 @@ __global__ void __launch_bounds__(kF8Threads, 1)
           }
         }
         __syncwarp();
+        if (lane == 0) mbar_arrive(&sempty_bar[pb]);
       }
 
       if (EPI == kEpiSwiGLU) {
@@ -379,7 +411,6 @@ __global__ void __launch_bounds__(kF8Threads, 1)
       } else {
         if (!ok) break;
         // Gates of the tile's tokens, then bf16 rows of both sub-tiles.
-        float *gates = sc;
         gates[lane] = lane < t.n_valid && args.row_scale ? __ldg(args.row_scale + t.row0 + lane)
                                                          : (lane < t.n_valid ? 1.f : 0.f);
         gates[32 + lane] = lane + 32 < t.n_valid && args.row_scale
