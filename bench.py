@@ -332,13 +332,28 @@ def near_tie_tokens(dm, x, W_r, b, ws):
     return int((gap <= 1e-4).sum().item())
 
 
-def decode_record(args, wt, device, rank, world):
+def decode_record(args, wt, device, rank, world, fp8_act=False):
     """The decode workload (T = 128) timed on the given expert weights, as its own record:
     ms per step, tokens/s, the dominant kernel against the HBM peak, the whole step's
-    fractions, per-stage times and clocks.  Every rank runs it (the max over ranks is taken)."""
+    fractions, per-stage times and clocks.  Every rank runs it (the max over ranks is taken).
+    With fp8_act the weights are first quantised to block-wise FP8 (outside the timed region)
+    and the layer runs with FP8 activations (E4M3 x E4M3 MMAs, moe_forward_fp8)."""
     w = WORKLOADS["decode"]
     x = make_tokens(w, device, seed=args.seed + rank)
-    dm = mb.dims(w.T, w.d, w.N, w.Z, w.K, w.I)
+    dm = mb.dims(w.T, w.d, w.N, w.Z, w.K, w.I, flags=mb.FP8_ACTIVATIONS if fp8_act else 0)
+    fw = None
+    if fp8_act:
+        log(f"[rank {rank}] quantising the expert weights to block-wise FP8 for the FP8 decode")
+        fw = mb.quantize_expert_weights_fp8(dm, wt["W_g"], wt["W_u"], wt["W_d"])
+
+    def forward(c, ev=None):
+        if fw is not None:
+            mb.moe_forward_fp8(dm, x, wt["W_r"], b, fw, y, c, ws, events=ev)
+        elif ev is None:
+            mb.moe_forward(dm, x, wt["W_r"], b, wt["W_g"], wt["W_u"], wt["W_d"], y, c, ws)
+        else:
+            mb.moe_forward_timed(dm, x, wt["W_r"], b, wt["W_g"], wt["W_u"], wt["W_d"], y, c, ws,
+                                 ev)
     ws = mb.alloc_workspace(dm, device)
     y = torch.empty((w.T, w.d), dtype=torch.bfloat16, device=device)
     b = wt["b"].clone()
@@ -353,7 +368,7 @@ def decode_record(args, wt, device, rank, world):
         for e in ev:
             e.record(stream)
     for i in range(args.warmup):
-        mb.moe_forward(dm, x, wt["W_r"], b, wt["W_g"], wt["W_u"], wt["W_d"], y, counts[i], ws)
+        forward(counts[i])
         mb.moe_bias_update(dm, counts[i], b, pid_state, params)
     torch.cuda.synchronize()
     if world > 1:
@@ -364,8 +379,7 @@ def decode_record(args, wt, device, rank, world):
     start.record(stream)
     for i in range(steps):
         c = counts[args.warmup + i]
-        mb.moe_forward_timed(dm, x, wt["W_r"], b, wt["W_g"], wt["W_u"], wt["W_d"], y, c, ws,
-                             events[i])
+        forward(c, events[i])
         mb.moe_bias_update(dm, c, b, pid_state, params)
     end.record(stream)
     torch.cuda.synchronize()
@@ -376,21 +390,28 @@ def decode_record(args, wt, device, rank, world):
         raise RuntimeError(f"device status {status:#x} after the decode steps")
     stage_ms = stage_durations(events)
     tot_flops, tot_bytes, (A_steps, U_steps, _) = step_work(
-        w, counts[args.warmup:].cpu().numpy())
+        w, counts[args.warmup:].cpu().numpy(), wb=1 if fp8_act else 2, ab=1 if fp8_act else 2)
     layer = layer_of(sum(tot_flops.values()), sum(tot_bytes.values()), ms, decode=True)
-    return {
+    rec = {
         "workload": w.name, "T": w.T, "steps": steps,
         "ms_per_step": round(ms / steps, 4),
         "value": round(job_throughput(world, w.T, steps, ms), 1), "unit": UNIT,
-        "roofline": roofline_of(w, stage_ms, tot_flops, tot_bytes),
+        "roofline": roofline_of(w, stage_ms, tot_flops, tot_bytes, fp8=fp8_act,
+                                fp8_act=fp8_act),
         "layer": layer,
         "stages_ms": {k: round(v / steps, 4) for k, v in stage_ms.items()},
         "mean_ffn_experts_per_token": round(float(np.mean(A_steps)) / w.T, 4),
         "distinct_ffn_experts": int(np.mean(U_steps)),
         "near_tie_tokens": near_tie_tokens(dm, x, wt["W_r"], b, ws),
         "clocks": clk,
-        "gpu_launches": LAUNCHES_PER_STEP * steps,
+        "gpu_launches": (LAUNCHES_PER_STEP + (1 if fp8_act else 0)) * steps,
     }
+    if fp8_act:
+        rec["variant"] = {"expert_weights": "fp8 e4m3, 128x128 blocks",
+                          "activations": "fp8 e4m3, 1x128 blocks (E4M3 x E4M3 MMAs)",
+                          "bytes_model": "1 byte per weight and per GEMM activation"}
+        del fw
+    return rec
 
 
 # ------------------------------------------------------------------------------ CPU oracle
@@ -560,8 +581,10 @@ def run_ours(args, rank, world, local_rank):
     layer["near_tie_tokens"] = near_tie_tokens(dm, x, wt["W_r"], b, ws)
     if not args.no_decode and w.name != "decode" and w.d == WORKLOADS["decode"].d and \
             w.N == WORKLOADS["decode"].N and w.I == WORKLOADS["decode"].I and not args.fp8:
-        # The second target's workload on the same expert weights (decode shares every one).
+        # The second target's workload on the same expert weights (decode shares every one),
+        # and the same with FP8 weights and activations read by the tensor cores.
         layer["decode"] = decode_record(args, wt, device, rank, world)
+        layer["decode_fp8"] = decode_record(args, wt, device, rank, world, fp8_act=True)
     if scmoe is not None:
         layer["scmoe"] = scmoe
 
@@ -636,6 +659,7 @@ def finish(args, w, world, rank, ms_max, routing, roof, layer, stage_ms, clk, e2
     A_steps, U_steps, load_ratio = routing
     near_ties = layer.pop("near_tie_tokens", None)
     decode = layer.pop("decode", None)
+    decode_fp8 = layer.pop("decode_fp8", None)
     result = {
         "metric": METRIC, "value": round(job_throughput(world, w.T, args.steps, ms_max), 1),
         "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -671,6 +695,8 @@ def finish(args, w, world, rank, ms_max, routing, roof, layer, stage_ms, clk, e2
     }
     if decode is not None:
         result["decode"] = decode
+    if decode_fp8 is not None:
+        result["decode_fp8_activations"] = decode_fp8
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         n = args.cpu_sample or default_sample(w)
         log(f"oracle CPU baseline on {n} sampled tokens ...")

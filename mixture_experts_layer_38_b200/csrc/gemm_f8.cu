@@ -48,7 +48,7 @@ constexpr int kF8BN = 64;                             // token rows per tile, at
 constexpr int kF8TileA = kBM * kF8BK;                 // 16 KB of codes per weight sub-tile
 constexpr int kF8Stage = 2 * kF8TileA + kF8BN * kF8BK;  // 40 KB
 constexpr int kF8Stages = 5;
-constexpr int kF8Parts = 4;                           // TMEM partial-sum buffers
+constexpr int kF8Parts = kTmemCols / (2 * kF8BN);     // TMEM partial-sum buffers
 constexpr int kF8PartCols = 2 * kF8BN;                // sub-tile 0 | sub-tile 1
 constexpr int kF8EpiWarps = 4;
 constexpr int kF8ScaleWarp = 2 + kF8EpiWarps;         // warp 6: block-scale loader
@@ -270,8 +270,10 @@ __global__ void __launch_bounds__(kF8Threads, 1)
         const float sw0 = __ldg(ws0 + kb);
         const float sw1 = t.has_a1 ? __ldg(ws1 + kb) : 0.f;
         const float *sx = args.act_scale + (long long)kb * args.rows + t.row0;
-        const float x0 = lane < t.n_valid ? __ldg(sx + lane) : 0.f;
-        const float x1 = lane + 32 < t.n_valid ? __ldg(sx + lane + 32) : 0.f;
+        float xs[kF8BN / 32];
+#pragma unroll
+        for (int i = 0; i < kF8BN / 32; ++i)
+          xs[i] = i * 32 + lane < t.n_valid ? __ldg(sx + i * 32 + lane) : 0.f;
         const int pb = (int)(n % kF8Parts);
         const uint32_t use = (uint32_t)(n / kF8Parts);
         if (!warp_wait(&sempty_bar[pb], (use & 1) ^ 1, abort_flag, wlim)) {
@@ -280,10 +282,11 @@ __global__ void __launch_bounds__(kF8Threads, 1)
           break;
         }
         float *slot = scale_ring + pb * kF8SlotFloats;
-        slot[lane] = x0 * sw0;
-        slot[32 + lane] = x1 * sw0;
-        slot[64 + lane] = x0 * sw1;
-        slot[96 + lane] = x1 * sw1;
+#pragma unroll
+        for (int i = 0; i < kF8BN / 32; ++i) {
+          slot[i * 32 + lane] = xs[i] * sw0;
+          slot[kF8BN + i * 32 + lane] = xs[i] * sw1;
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(&sfull_bar[pb]);
       }
@@ -333,7 +336,7 @@ __global__ void __launch_bounds__(kF8Threads, 1)
 #pragma unroll
             for (int j4 = 0; j4 < 8; ++j4) {
               const float4 s0 = reinterpret_cast<const float4 *>(sc)[c * 8 + j4];
-              const float4 s1 = reinterpret_cast<const float4 *>(sc + 64)[c * 8 + j4];
+              const float4 s1 = reinterpret_cast<const float4 *>(sc + kF8BN)[c * 8 + j4];
               const int j = c * 32 + j4 * 4;
               acc0[j] = fmaf(__uint_as_float(p0[j4 * 4]), s0.x, acc0[j]);
               acc0[j + 1] = fmaf(__uint_as_float(p0[j4 * 4 + 1]), s0.y, acc0[j + 1]);
@@ -354,13 +357,14 @@ __global__ void __launch_bounds__(kF8Threads, 1)
         // h, then its E4M3 codes: the four warps agree on stopping before their barriers.
         if (lane == 0 && (!ok || *abort_flag)) *stop_flag = 1;
 #pragma unroll
-        for (int j = 0; j < kF8BN; ++j) acc0[j] = silu(acc0[j]) * acc1[j];
-#pragma unroll
         for (int c = 0; c < kF8BN / 32; ++c) {
           if (c < chunks) {
             float v[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = acc0[c * 32 + j];
+            for (int j = 0; j < 32; ++j) {
+              acc0[c * 32 + j] = silu(acc0[c * 32 + j]) * acc1[c * 32 + j];
+              v[j] = acc0[c * 32 + j];
+            }
             colmax[ew * kF8BN + c * 32 + lane] = warp_column_absmax(v, lane);
           }
         }
@@ -400,7 +404,7 @@ __global__ void __launch_bounds__(kF8Threads, 1)
         __syncwarp();
         uint8_t *out = reinterpret_cast<uint8_t *>(args.out);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < kF8BN / 16; ++i) {
           const int p = i * 32 + lane, j = p >> 1, half = p & 1;
           if (j < t.n_valid)
             *reinterpret_cast<uint4 *>(out + (long long)(t.row0 + j) * args.out_ld + t.m0 +
@@ -411,11 +415,12 @@ __global__ void __launch_bounds__(kF8Threads, 1)
       } else {
         if (!ok) break;
         // Gates of the tile's tokens, then bf16 rows of both sub-tiles.
-        gates[lane] = lane < t.n_valid && args.row_scale ? __ldg(args.row_scale + t.row0 + lane)
-                                                         : (lane < t.n_valid ? 1.f : 0.f);
-        gates[32 + lane] = lane + 32 < t.n_valid && args.row_scale
-                               ? __ldg(args.row_scale + t.row0 + 32 + lane)
-                               : (lane + 32 < t.n_valid ? 1.f : 0.f);
+#pragma unroll
+        for (int i = 0; i < kF8BN / 32; ++i) {
+          const int j = i * 32 + lane;
+          gates[j] = j >= t.n_valid ? 0.f : (args.row_scale ? __ldg(args.row_scale + t.row0 + j)
+                                                            : 1.f);
+        }
         __syncwarp();
         uint32_t *stg = reinterpret_cast<uint32_t *>(stage_bytes);
         uint16_t *out = reinterpret_cast<uint16_t *>(args.out);
