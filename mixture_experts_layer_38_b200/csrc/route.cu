@@ -171,12 +171,14 @@ __global__ void __launch_bounds__(kBlockThreads, kPerThread <= 3 ? 4 : 3)
   }
 }
 
-// Pools of up to 256 experts: one warp per token (8 tokens per block), lane i holding experts
-// i, i + 32, ...; the same keys and K+1 argmax rounds as above, with warp shuffles only, so a
-// small pool does not leave most of a 256-thread block idle.
-constexpr int kWarpPer = 8;  // experts per lane: E <= 256
-
-__global__ void __launch_bounds__(256)
+// One warp per token (8 tokens per block), lane i holding experts i, i + 32, ... (kWarpPer of
+// them: E <= 32 * kWarpPer); the same keys and K+1 argmax rounds as above, with warp shuffles
+// only.  Used for small pools (a 96-expert pool would leave most of a 256-thread block idle)
+// and for large batches of any pool (no block barrier per round, about a fifth of the block
+// kernel's instructions per token); a small batch of a large pool keeps the block kernel,
+// whose 8 warps per token spread a short batch over more SMs.
+template <int kWarpPer>
+__global__ void __launch_bounds__(256, kWarpPer <= 8 ? 1 : 2)
     route_topk_warp_kernel(const float *__restrict__ logits, int splits, int T, int E, int ld,
                            int K, const float *__restrict__ b, bool renormalize,
                            int32_t *__restrict__ topk_idx, float *__restrict__ topk_gate,
@@ -209,21 +211,33 @@ __global__ void __launch_bounds__(256)
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
-  uint64_t key[kWarpPer];
+  // Scores as order-preserving 32-bit patterns (0 = taken or not an expert; every real score
+  // maps above 0); the id of slot j of this lane is lane + 32 j, so the 64-bit key of the
+  // selection order (score, then the lower id) is formed only for the warp-wide maximum.
+  uint32_t sk[kWarpPer];
 #pragma unroll
   for (int j = 0; j < kWarpPer; ++j) {
     const int e = lane + 32 * j;
     p[j] = __fdiv_rn(p[j], z);
-    key[j] = (e < E) ? score_key(__fadd_rn(p[j], __ldg(b + e)), e) : 0ull;
+    sk[j] = (e < E) ? (uint32_t)(score_key(__fadd_rn(p[j], __ldg(b + e)), e) >> 32) : 0u;
   }
   const int rounds = K < E ? K + 1 : K;
   int my_id = 0x7fffffff;  // lane k keeps the k-th selected expert
   float my_p = 0.f, s_k1 = 0.f, s_k = 0.f;
   for (int k = 0; k < rounds; ++k) {
-    uint64_t best = key[0];
+    uint32_t bs = sk[0];
+    int bj = 0;
 #pragma unroll
-    for (int j = 1; j < kWarpPer; ++j) best = key[j] > best ? key[j] : best;
-    best = warp_max_u64(best);
+    for (int j = 1; j < kWarpPer; ++j) {  // strict: among equal scores the lower id (lower j)
+      if (sk[j] > bs) {
+        bs = sk[j];
+        bj = j;
+      }
+    }
+    const uint64_t mine = bs == 0u ? 0ull
+                                   : ((uint64_t)bs << 32) |
+                                         (0xffffffffu - (uint32_t)(lane + 32 * bj));
+    const uint64_t best = warp_max_u64(mine);
     if (best == 0ull) {  // nothing left that is selectable (non-finite scores): flag, skip
       if (lane == 0) record_status(status, MOE_DEV_BAD_EXPERT);
       continue;
@@ -231,11 +245,13 @@ __global__ void __launch_bounds__(256)
     const int id = (int)(0xffffffffu - (uint32_t)(best & 0xffffffffu));
     const int owner = id & 31, jo = id >> 5;
     float pv = 0.f;
+    if (lane == owner) {
 #pragma unroll
-    for (int j = 0; j < kWarpPer; ++j) {
-      if (j == jo && lane == owner) {
-        pv = p[j];
-        key[j] = 0ull;
+      for (int j = 0; j < kWarpPer; ++j) {
+        if (j == jo) {
+          pv = p[j];
+          sk[j] = 0u;
+        }
       }
     }
     pv = __shfl_sync(0xffffffffu, pv, owner);
@@ -266,6 +282,9 @@ __global__ void __launch_bounds__(256)
   }
   if (gap != nullptr && lane == 0) gap[t] = (K < E) ? __fsub_rn(s_k1, s_k) : INFINITY;
 }
+
+// Tokens from which a pool of more than 256 experts goes to the warp-per-token kernel.
+constexpr int kWarpTopkMinTokens = 2048;
 
 }  // namespace
 
@@ -299,8 +318,18 @@ cudaError_t launch_route_topk(const float *logits, int splits, int T, int E, int
                               float *topk_gate, float *gap, int *status, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
   const int ld = (E + 3) & ~3;
-  if (E <= 32 * kWarpPer)
-    route_topk_warp_kernel<<<(T + 7) / 8, 256, 0, stream>>>(
+  const int blocks = (T + 7) / 8;
+  if (E <= 256)
+    route_topk_warp_kernel<8><<<blocks, 256, 0, stream>>>(
+        logits, splits, T, E, ld, K, b, renormalize, topk_idx, topk_gate, gap, status);
+  else if (T >= kWarpTopkMinTokens && E <= 512)
+    route_topk_warp_kernel<16><<<blocks, 256, 0, stream>>>(
+        logits, splits, T, E, ld, K, b, renormalize, topk_idx, topk_gate, gap, status);
+  else if (T >= kWarpTopkMinTokens && E <= 768)
+    route_topk_warp_kernel<24><<<blocks, 256, 0, stream>>>(
+        logits, splits, T, E, ld, K, b, renormalize, topk_idx, topk_gate, gap, status);
+  else if (T >= kWarpTopkMinTokens)
+    route_topk_warp_kernel<32><<<blocks, 256, 0, stream>>>(
         logits, splits, T, E, ld, K, b, renormalize, topk_idx, topk_gate, gap, status);
   else if (E <= 3 * kBlockThreads)
     route_topk_block_kernel<3><<<T, kBlockThreads, 0, stream>>>(
