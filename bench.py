@@ -459,7 +459,8 @@ def run_ours(args, rank, world, local_rank):
     x = make_tokens(w, device, seed=args.seed + rank)
     dm = mb.dims(w.T, w.d, w.N, w.Z, w.K, w.I,
                  flags=(mb.RENORMALIZE_GATES if args.renormalize_gates else 0) |
-                 (mb.FP8_ACTIVATIONS if args.fp8_activations else 0))
+                 (mb.FP8_ACTIVATIONS if args.fp8_activations else 0) |
+                 (mb.FUSED_COMBINE if args.fused_combine else 0))
     ws = mb.alloc_workspace(dm, device)
     y = torch.empty((w.T, w.d), dtype=torch.bfloat16, device=device)
     b = wt["b"].clone()
@@ -679,6 +680,7 @@ def finish(args, w, world, rank, ms_max, routing, roof, layer, stage_ms, clk, e2
                         "expert_weights": "fp8 e4m3, 128x128 blocks" if args.fp8 else "bf16",
                         "activations": "fp8 e4m3, 1x128 blocks (E4M3 x E4M3 MMAs)"
                                        if args.fp8_activations else "bf16",
+                        "fused_combine": bool(args.fused_combine),
                         "scmoe_dense_ffn": args.scmoe or None},
             "mean_ffn_experts_per_token": round(float(np.mean(A_steps)) / w.T, 4),
             "distinct_ffn_experts": int(np.mean(U_steps)),
@@ -773,6 +775,8 @@ def main():
     ap.add_argument("--fp8-activations", action="store_true",
                     help="variant (with --fp8): E4M3 activations too, 1x128 blocks, read by "
                          "E4M3 x E4M3 tensor-core MMAs")
+    ap.add_argument("--fused-combine", action="store_true",
+                    help="variant: the combine fused into the down projection's epilogue")
     ap.add_argument("--balance-gamma", type=float, default=0.0,
                     help="variant: step of the per-expert balancing term after the PID step")
     args = ap.parse_args()
@@ -780,6 +784,8 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.fp8_activations and not args.fp8:
         ap.error("--fp8-activations needs --fp8")
+    if args.fused_combine and args.fp8:
+        ap.error("--fused-combine runs with bf16 weights only")
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))

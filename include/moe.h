@@ -53,8 +53,8 @@ typedef struct {
     int32_t Z; /* zero-computation experts (ids N .. N+Z-1) */
     int32_t K; /* experts selected per token */
     int32_t I; /* intermediate width of each SwiGLU FFN expert */
-    uint32_t flags; /* variant switches (MOE_RENORMALIZE_GATES, MOE_FP8_ACTIVATIONS); 0 = the
-                       layer as defined */
+    uint32_t flags; /* variant switches (MOE_RENORMALIZE_GATES, MOE_FP8_ACTIVATIONS,
+                       MOE_FUSED_COMBINE); 0 = the layer as defined */
 } moe_dims;
 
 /* Gates renormalised over the selected set: g_i = p_i / sum of p over the K selected experts
@@ -72,6 +72,18 @@ typedef struct {
  * (MOE_ERR_SHAPE otherwise); the codes and scales of x_perm and h live in the workspace scratch
  * (moe_scratch_size grows by about T*K*(d + I)*1.03 bytes). */
 #define MOE_FP8_ACTIVATIONS 2u
+
+/* The combine fused into the down projection, for moe_forward / moe_forward_timed with bf16
+ * weights only (every other entry point returns MOE_ERR_ARG when it is set): the down
+ * projection's epilogue counts, per token and feature block, the FFN rows it has stored; the
+ * tile completing a token's count sums that block of y_t from the token's rows in slot order
+ * with the combine's arithmetic, so y is bit-identical to the unfused layer whichever tile
+ * finishes last; tokens without an FFN slot are written by a zero-only combine pass.  The down
+ * projection then runs on single CTAs, and the workspace grows by T * 4 * ceil(d / 256) * 4
+ * bytes of counters (set by the call).  An optional variant after the CSDN codearts article
+ * on LongCat-Flash, §二、训练优化 (tiles accumulated in a deterministic order, the fp32 addition
+ * fused into the GEMM epilogue instead of written back and re-read). */
+#define MOE_FUSED_COMBINE 4u
 
 /* PID gains and set-point: target = desired mean number of FFN experts per token.
  * balance_gamma: step of the per-expert balancing term (see moe_bias_update); 0 = off. */

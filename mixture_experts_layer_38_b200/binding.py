@@ -105,6 +105,7 @@ def lib():
 
 RENORMALIZE_GATES = 1  # MOE_RENORMALIZE_GATES
 FP8_ACTIVATIONS = 2  # MOE_FP8_ACTIVATIONS
+FUSED_COMBINE = 4  # MOE_FUSED_COMBINE
 
 
 def dims(T, d, N, Z, K, I, flags=0) -> Dims:

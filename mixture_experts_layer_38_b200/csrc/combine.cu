@@ -24,7 +24,7 @@ __global__ void __launch_bounds__(kCombineThreads)
     combine_kernel(const uint4 *__restrict__ x, const uint4 *__restrict__ y_perm,
                    const int32_t *__restrict__ topk_idx, const float *__restrict__ topk_gate,
                    const int32_t *__restrict__ slot_pos, int T, int d16, int N, int K, int rows,
-                   uint4 *__restrict__ y, int *status) {
+                   uint4 *__restrict__ y, int *status, bool zero_only) {
   __shared__ int s_pos[kMaxK];
   __shared__ float s_zsum;
   __shared__ int s_nffn;
@@ -50,30 +50,26 @@ __global__ void __launch_bounds__(kCombineThreads)
   __syncthreads();
   const float zsum = s_zsum;
   const int nffn = s_nffn;
+  if (zero_only && nffn > 0) return;  // written by the combine fused into the down projection
   for (int i = threadIdx.x; i < d16; i += kCombineThreads) {
     float acc[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-    for (int n = 0; n < nffn; ++n) {
-      const uint4 v = __ldg(y_perm + (long long)s_pos[n] * d16 + i);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        acc[2 * j] += __uint_as_float(w[j] << 16);
-        acc[2 * j + 1] += __uint_as_float(w[j] & 0xffff0000u);
-      }
-    }
-    const uint4 xv = __ldg(x + (long long)t * d16 + i);
-    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-    uint32_t o[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float lo = acc[2 * j] + zsum * __uint_as_float(xw[j] << 16);
-      const float hi = acc[2 * j + 1] + zsum * __uint_as_float(xw[j] & 0xffff0000u);
-      o[j] = pack_bf16x2(lo, hi);
-    }
-    y[(long long)t * d16 + i] = make_uint4(o[0], o[1], o[2], o[3]);
+    for (int n = 0; n < nffn; ++n) combine_add8(acc, __ldg(y_perm + (long long)s_pos[n] * d16 + i));
+    y[(long long)t * d16 + i] = combine_finish8(acc, zsum, __ldg(x + (long long)t * d16 + i));
   }
+}
+
+// Counters of the combine fused into the down projection: every feature block of token t
+// starts at t's number of FFN slots.
+__global__ void __launch_bounds__(256)
+    combine_counters_kernel(const int32_t *__restrict__ topk_idx, int T, int K, int N,
+                            int blocks, int *__restrict__ count) {
+  const int t = blockIdx.x * 256 + threadIdx.x;
+  if (t >= T) return;
+  int nffn = 0;
+  for (int k = 0; k < K; ++k) nffn += __ldg(topk_idx + (long long)t * K + k) < N;
+  for (int b = 0; b < blocks; ++b) count[(long long)t * blocks + b] = nffn;
 }
 
 __global__ void __launch_bounds__(256)
@@ -118,11 +114,20 @@ __global__ void __launch_bounds__(256)
 
 cudaError_t launch_combine(const uint16_t *x, const uint16_t *y_perm, const int32_t *topk_idx,
                            const float *topk_gate, const int32_t *slot_pos, int T, int d, int N,
-                           int K, int rows, uint16_t *y, int *status, cudaStream_t stream) {
+                           int K, int rows, uint16_t *y, int *status, cudaStream_t stream,
+                           bool zero_only) {
   if (T == 0) return cudaSuccess;
   combine_kernel<<<T, kCombineThreads, 0, stream>>>(
       reinterpret_cast<const uint4 *>(x), reinterpret_cast<const uint4 *>(y_perm), topk_idx,
-      topk_gate, slot_pos, T, d / 8, N, K, rows, reinterpret_cast<uint4 *>(y), status);
+      topk_gate, slot_pos, T, d / 8, N, K, rows, reinterpret_cast<uint4 *>(y), status,
+      zero_only);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine_counters(const int32_t *topk_idx, int T, int K, int N, int blocks,
+                                    int *count, cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  combine_counters_kernel<<<(T + 255) / 256, 256, 0, stream>>>(topk_idx, T, K, N, blocks, count);
   return cudaGetLastError();
 }
 

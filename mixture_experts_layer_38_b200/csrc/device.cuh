@@ -330,6 +330,32 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// ---------------------------------------------------------------- combine arithmetic
+// One 16-byte piece (8 bf16 features) of the layer's combine, shared by the combine kernel and
+// the combine fused into the down projection so both give the same bits: the token's FFN rows
+// are added in slot order into fp32 (combine_add8), then y = sum + zsum * x, one bf16 rounding.
+__device__ __forceinline__ void combine_add8(float (&acc)[8], uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    acc[2 * j] += __uint_as_float(w[j] << 16);
+    acc[2 * j + 1] += __uint_as_float(w[j] & 0xffff0000u);
+  }
+}
+
+__device__ __forceinline__ uint4 combine_finish8(const float (&acc)[8], float zsum, uint4 xv) {
+  const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float lo = __fmaf_rn(zsum, __uint_as_float(xw[j] << 16), acc[2 * j]);
+    const float hi = __fmaf_rn(zsum, __uint_as_float(xw[j] & 0xffff0000u), acc[2 * j + 1]);
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    o[j] = *reinterpret_cast<uint32_t *>(&v);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 // ---------------------------------------------------------------- misc
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);

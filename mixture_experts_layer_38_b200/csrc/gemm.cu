@@ -112,7 +112,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs &a, const Tile &t,
     for (int j = 0; j < 32; ++j) h[j] = silu(__uint_as_float(g[j])) * __uint_as_float(u[j]);
     store_rows_bf16(reinterpret_cast<uint16_t *>(a.out), a.out_ld, t.row0, tok0, t.n_valid,
                     t.m0 + q * 32, a.M, lane, h, reinterpret_cast<uint32_t *>(stage));
-  } else if (EPI == kEpiGated) {
+  } else if (EPI == kEpiGated || EPI == kEpiGatedCombine) {
     // The chunk's 32 gates, read by every lane as broadcast vector loads from the warp's
     // staging area (one store per lane, eight loads) instead of 32 shuffles.
     const int tok = tok0 + lane;
@@ -170,6 +170,95 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs &a, const Tile &t,
         }
       }
     }
+  }
+}
+
+// ------------------------------------------------------------------ combine fused into GEMM2
+// kEpiGatedCombine (the MoE layer's combine in the down projection's epilogue, deterministic):
+// warp q of a tile owns feature block (tile's m-range, q) = features m0 + q*32 + [0, 32) and
+// m0 + 128 + q*32 + [0, 32).  Each token's counter of each block starts at the token's number of
+// FFN slots (launch_combine_counters).  After storing a 32-token chunk of y_perm rows, the warp
+// makes the stores visible device-wide and counts one arrival down per token; the arrival that
+// reaches zero belongs to the last tile holding one of the token's rows for that block, and that
+// warp then sums the block of y for the token from y_perm in slot order -- the combine kernel's
+// arithmetic (combine_add8 / combine_finish8), so the result does not depend on which tile
+// finishes last.  Tokens with no FFN slot are left to launch_combine's zero-only pass.
+
+// Counts the arrivals of the tile's tokens (after all of the warp's stores of the tile, one
+// fence): one atomic per token, all issued before any result is used.  fin[c] gets the lanes
+// (tokens c * 32 + lane) this warp completes.
+template <int NC>
+__device__ __forceinline__ void combine_count(const GemmArgs &a, const Tile &t, int chunks, int q,
+                                              int lane, uint32_t (&fin)[NC]) {
+  __threadfence();  // this lane's y_perm stores before its arrivals
+  __syncwarp();
+  const int blk = (t.m0 / (2 * kBM)) * 4 + q;
+  int old[NC];
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+    old[c] = 0;
+    const int j = c * 32 + lane;
+    if (c < chunks && j < t.n_valid) {
+      const long long tok = __ldg(a.cmb_perm_tok + t.row0 + j);
+      old[c] = atomicSub(a.cmb_count + tok * a.cmb_blocks + blk, 1);
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < NC; ++c) fin[c] = __ballot_sync(0xffffffffu, old[c] == 1);
+}
+
+// Sums the completed tokens' blocks of y, four tokens at a time (eight lanes, 16 bytes each).
+__device__ __forceinline__ void combine_finish(const GemmArgs &a, const Tile &t, int tok0,
+                                               uint32_t fin, int q, int lane) {
+  __threadfence();  // the other tiles' rows, whose arrivals preceded ours, are visible
+  const int g = lane >> 3, i = lane & 7;
+  const int f = t.m0 + (i < 4 ? 0 : kBM) + q * 32 + (i & 3) * 8;
+  const uint16_t *y_perm = reinterpret_cast<const uint16_t *>(a.out);
+  while (fin != 0u) {
+    uint32_t m = fin;
+    for (int s = 0; s < g && m != 0u; ++s) m &= m - 1;  // the g-th lowest remaining token
+    if (m != 0u && f < a.M) {
+      const long long tok = __ldg(a.cmb_perm_tok + t.row0 + tok0 + __ffs(m) - 1);
+      float acc[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+      float zsum = 0.f;
+      // Eight slots at a time: their loads are independent, the sums stay in slot order.
+      constexpr int kB = 8;
+      for (int k0 = 0; k0 < a.cmb_K; k0 += kB) {
+        int e[kB], r[kB];
+        float gv[kB];
+        uint4 v[kB];
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+          const long long slot = tok * a.cmb_K + k0 + u;
+          const bool in = k0 + u < a.cmb_K;
+          e[u] = in ? __ldg(a.cmb_idx + slot) : a.cmb_N;
+          r[u] = in ? __ldg(a.cmb_slot + slot) : 0;
+          gv[u] = in ? __ldg(a.cmb_gate + slot) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+          v[u] = make_uint4(0u, 0u, 0u, 0u);
+          if (e[u] < a.cmb_N && r[u] >= 0 && r[u] < a.rows)
+            v[u] = __ldcg(reinterpret_cast<const uint4 *>(y_perm + (long long)r[u] * a.out_ld +
+                                                          f));
+        }
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+          if (k0 + u >= a.cmb_K) break;
+          if (e[u] >= a.cmb_N)
+            zsum += gv[u];
+          else if (r[u] >= 0 && r[u] < a.rows)
+            combine_add8(acc, v[u]);
+          else
+            record_status(a.status, MOE_DEV_BAD_ROWS);
+        }
+      }
+      const uint4 xv = __ldg(reinterpret_cast<const uint4 *>(a.cmb_x + tok * a.M + f));
+      *reinterpret_cast<uint4 *>(a.cmb_y + tok * a.M + f) = combine_finish8(acc, zsum, xv);
+    }
+    for (int s = 0; s < 4 && fin != 0u; ++s) fin &= fin - 1;
   }
 }
 
@@ -509,11 +598,27 @@ __global__ void __launch_bounds__(Cfg<BN, WQ, GATHER>::kThreads, 1)
       tc_fence_after();
       const uint32_t tcol = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * (2 * BN);
       const int chunks = (t.n_valid + 31) / 32;
-      for (int c = group; c < chunks; c += kEpiGroups)
-        epilogue_chunk<EPI, BN>(args, t, tcol + c * 32, c, q, lane, stage);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty_bar[buf]);
+      if (EPI == kEpiGatedCombine) {
+        // Stores and arrivals first, then the accumulator is released, then the sums.
+        static_assert(EPI != kEpiGatedCombine || kEpiGroups == 1, "one warp per quarter");
+        uint32_t fin[BN / 32];
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c)
+          if (c < chunks) epilogue_chunk<EPI, BN>(args, t, tcol + c * 32, c, q, lane, stage);
+        combine_count(args, t, chunks, q, lane, fin);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty_bar[buf]);
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c)
+          if (c < chunks && fin[c] != 0u) combine_finish(args, t, c * 32, fin[c], q, lane);
+      } else {
+        for (int c = group; c < chunks; c += kEpiGroups)
+          epilogue_chunk<EPI, BN>(args, t, tcol + c * 32, c, q, lane, stage);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty_bar[buf]);
+      }
     }
   }
 
@@ -992,6 +1097,10 @@ cudaError_t launch_bn(int epi, const GemmArgs &args_in, int grid, cudaStream_t s
     case kEpiGated:
       grouped_gemm_kernel<kEpiGated, BN, false, false><<<grid, threads, smem, stream>>>(args);
       break;
+    case kEpiGatedCombine:
+      grouped_gemm_kernel<kEpiGatedCombine, BN, false, false>
+          <<<grid, threads, smem, stream>>>(args);
+      break;
     default:
       grouped_gemm_kernel<kEpiF32, BN, false, false><<<grid, threads, smem, stream>>>(args);
       break;
@@ -1008,6 +1117,8 @@ cudaError_t gemm_prepare(int device) {
   if ((e = prepare_dual<kEpiGated>(device)) != cudaSuccess) return e;
   if ((e = set_smem_limit<kEpiSwiGLU, 128>()) != cudaSuccess) return e;
   if ((e = set_smem_limit<kEpiGated, 128>()) != cudaSuccess) return e;
+  if ((e = set_smem_limit<kEpiGatedCombine, 128>()) != cudaSuccess) return e;
+  if ((e = set_smem_limit<kEpiGatedCombine, 256>()) != cudaSuccess) return e;
   if ((e = set_smem_limit<kEpiF32, 128>()) != cudaSuccess) return e;
   if ((e = set_smem_limit<kEpiSwiGLU, 256>()) != cudaSuccess) return e;
   if ((e = set_smem_limit<kEpiGated, 256>()) != cudaSuccess) return e;

@@ -13,7 +13,9 @@ namespace moe {
 enum EpiKind : int {
   kEpiSwiGLU = 0,  // h = silu(A0 x) * (A1 x)           -> bf16 [rows, M]
   kEpiGated = 1,   // y = row_scale[r] * (A x)          -> bf16 [rows, M]
-  kEpiF32 = 2      // logits (split-K partials)         -> fp32 [splits][rows, M]
+  kEpiF32 = 2,     // logits (split-K partials)         -> fp32 [splits][rows, M]
+  kEpiGatedCombine = 3  // kEpiGated, then the layer's combine fused in: the last tile to store
+                        // a token's rows of a feature block sums that block of y (gemm.cu)
 };
 
 struct GemmArgs {
@@ -58,6 +60,17 @@ struct GemmArgs {
   // E4M3 codes (out, [rows, M] bytes) and their scales to out_scale[(f / 128) * rows + r].
   const float *act_scale;
   float *out_scale;
+  // kEpiGatedCombine: the combine of the MoE layer (see launch_combine) fused into the down
+  // projection.  cmb_count [T, cmb_blocks] holds each token's FFN-slot count at launch
+  // (launch_combine_counters); cmb_blocks = 4 * m-tiles.
+  const uint16_t *cmb_x;        // [T, M] token inputs
+  const int32_t *cmb_perm_tok;  // [rows] token of each grouped row
+  const int32_t *cmb_idx;       // [T, K] selected expert ids, ascending
+  const float *cmb_gate;        // [T, K] gates
+  const int32_t *cmb_slot;      // [T, K] grouped row of each FFN slot
+  int *cmb_count;
+  uint16_t *cmb_y;              // [T, M] layer output
+  int cmb_K, cmb_N, cmb_blocks;
 };
 
 // Grouped GEMM block: warp 0 issues TMA loads, warp 1 allocates TMEM and issues MMAs, and
@@ -127,9 +140,14 @@ cudaError_t launch_dispatch(const uint16_t *x, const int32_t *topk_idx, const fl
                             int num_sms, cudaStream_t stream);
 
 // ------------------------------------------------------------------ combine and PID
+// zero_only: write only the tokens with no FFN slot (the others come from the fused combine).
 cudaError_t launch_combine(const uint16_t *x, const uint16_t *y_perm, const int32_t *topk_idx,
                            const float *topk_gate, const int32_t *slot_pos, int T, int d, int N,
-                           int K, int rows, uint16_t *y, int *status, cudaStream_t stream);
+                           int K, int rows, uint16_t *y, int *status, cudaStream_t stream,
+                           bool zero_only = false);
+// Fused combine: count[t * blocks + b] = number of FFN slots of token t, for every block b.
+cudaError_t launch_combine_counters(const int32_t *topk_idx, int T, int K, int N, int blocks,
+                                    int *count, cudaStream_t stream);
 // PID step on the FFN biases, then (gamma != 0) the per-expert balancing term.
 cudaError_t launch_pid(const int32_t *counts, int N, int K, int T, float *b, float *state,
                        float target, float kp, float ki, float kd, float gamma,

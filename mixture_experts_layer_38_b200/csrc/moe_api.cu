@@ -166,7 +166,8 @@ bool dims_ok(const moe_dims *d) {
   if (d->K < 1 || d->K > kMaxK || d->K > E) return false;
   if ((long long)d->T * d->K >= (1ll << 31)) return false;
   if ((long long)d->N * d->I >= (1ll << 31) || (long long)d->N * d->d >= (1ll << 31)) return false;
-  if ((d->flags & ~(MOE_RENORMALIZE_GATES | MOE_FP8_ACTIVATIONS)) != 0) return false;
+  if ((d->flags & ~(MOE_RENORMALIZE_GATES | MOE_FP8_ACTIVATIONS | MOE_FUSED_COMBINE)) != 0)
+    return false;
   // FP8 activations are scaled per 128 channels (and need FP8 weights, whose blocks are 128).
   if ((d->flags & MOE_FP8_ACTIVATIONS) && (d->d % 128 != 0 || d->I % 128 != 0)) return false;
   return true;
@@ -176,6 +177,9 @@ bool dims_ok(const moe_dims *d) {
 bool fp8_dims_ok(const moe_dims &d) { return d.d % 128 == 0 && d.I % 128 == 0; }
 
 bool fp8_act(const moe_dims &d) { return (d.flags & MOE_FP8_ACTIVATIONS) != 0; }
+bool fused_combine(const moe_dims &d) { return (d.flags & MOE_FUSED_COMBINE) != 0; }
+// Feature blocks of the fused combine: four per 256-feature m-tile of the down projection.
+int combine_blocks(const moe_dims &d) { return 4 * ((d.d + 255) / 256); }
 
 int router_splits(const moe_dims &d) {
   const int E = d.N + d.Z;
@@ -193,7 +197,7 @@ struct Layout {
   int epad;
   size_t status, logits, chunk, xq, sx, hq, sh, scratch_end;
   size_t topk_idx, topk_gate, gap, counts, offsets, perm_tok, perm_gate, slot_pos;
-  size_t x_perm, h, y_perm, total;
+  size_t x_perm, h, y_perm, cmb_count, total;
 };
 
 Layout layout_of(const moe_dims &d) {
@@ -229,6 +233,7 @@ Layout layout_of(const moe_dims &d) {
   L.x_perm = take(rows * (size_t)d.d * 2);
   L.h = take(rows * (size_t)d.I * 2);
   L.y_perm = take(rows * (size_t)d.d * 2);
+  if (d.flags & MOE_FUSED_COMBINE) L.cmb_count = take(T * (size_t)combine_blocks(d) * 4);
   L.total = off;
   return L;
 }
@@ -330,7 +335,8 @@ int do_expert_ffn(const moe_dims &d, const DeviceInfo &di, const Layout &L,
                   const moe_bf16 *W_g, const moe_bf16 *W_u, const moe_bf16 *W_d, moe_bf16 *h,
                   moe_bf16 *y_perm, void *ws, cudaStream_t stream,
                   void *const *events = nullptr, const moe_bf16 *x = nullptr,
-                  const int32_t *perm_tok = nullptr, const Fp8Weights *fw = nullptr) {
+                  const int32_t *perm_tok = nullptr, const Fp8Weights *fw = nullptr,
+                  const GemmArgs *cmb = nullptr) {
   if (d.T == 0 || d.N == 0) return record(events, 4, stream);
   const uint64_t rows = (uint64_t)d.T * d.K;
   int *status = at<int>(ws, L.status);
@@ -413,6 +419,22 @@ int do_expert_ffn(const moe_dims &d, const DeviceInfo &di, const Layout &L,
     down.scale_a1 = fw->s_d;
     down.scale_ld = d.I / 128;
     return to_status(launch_grouped_gemm_fp8(kEpiGated, down, di.sms, stream));
+  }
+  if (cmb != nullptr) {  // the combine fused into the down projection (single CTAs)
+    down.cmb_x = cmb->cmb_x;
+    down.cmb_perm_tok = cmb->cmb_perm_tok;
+    down.cmb_idx = cmb->cmb_idx;
+    down.cmb_gate = cmb->cmb_gate;
+    down.cmb_slot = cmb->cmb_slot;
+    down.cmb_count = cmb->cmb_count;
+    down.cmb_y = cmb->cmb_y;
+    down.cmb_K = cmb->cmb_K;
+    down.cmb_N = cmb->cmb_N;
+    down.cmb_blocks = cmb->cmb_blocks;
+    if (launch_combine_counters(down.cmb_idx, d.T, d.K, d.N, down.cmb_blocks, down.cmb_count,
+                                stream) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return to_status(launch_grouped_gemm(kEpiGatedCombine, down, di.sms, tile_tokens, stream));
   }
   if (dual) return to_status(launch_grouped_gemm_dual(kEpiGated, down, di.dual_pairs, stream));
   return to_status(launch_grouped_gemm(kEpiGated, down, di.sms, tile_tokens, stream));
@@ -566,6 +588,7 @@ int moe_expert_ffn(const moe_dims *dims, const moe_bf16 *x_perm, const int32_t *
   MOE_REQUIRE(dims != nullptr, MOE_ERR_ARG);
   MOE_REQUIRE(dims_ok(dims), MOE_ERR_SHAPE);
   MOE_REQUIRE(!fp8_act(*dims), MOE_ERR_ARG);  // FP8 activations need FP8 weights
+  MOE_REQUIRE(!fused_combine(*dims), MOE_ERR_ARG);  // moe_forward only
   MOE_CHECK_TOKEN_PTR(x_perm, dims->T);
   MOE_CHECK_PTR(offsets);
   MOE_CHECK_TOKEN_PTR(perm_gate, dims->T);
@@ -590,7 +613,7 @@ int moe_expert_ffn_gather(const moe_dims *dims, const moe_bf16 *x, const int32_t
                           moe_bf16 *y_perm, void *ws, size_t ws_bytes, void *stream) {
   MOE_REQUIRE(dims != nullptr, MOE_ERR_ARG);
   MOE_REQUIRE(dims_ok(dims), MOE_ERR_SHAPE);
-  MOE_REQUIRE(!fp8_act(*dims), MOE_ERR_ARG);
+  MOE_REQUIRE(!fp8_act(*dims) && !fused_combine(*dims), MOE_ERR_ARG);
   MOE_CHECK_TOKEN_PTR(x, dims->T);
   MOE_CHECK_TOKEN_PTR(perm_tok, dims->T);
   MOE_CHECK_PTR(offsets);
@@ -754,6 +777,7 @@ int forward_impl(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *W_r, c
     MOE_CHECK_PTR(W_d);
   } else {
     MOE_REQUIRE(fp8_dims_ok(*dims), MOE_ERR_SHAPE);
+    MOE_REQUIRE(!fused_combine(*dims), MOE_ERR_ARG);  // bf16 weights only
     MOE_CHECK_PTR(fw->q_g);
     MOE_CHECK_PTR(fw->q_u);
     MOE_CHECK_PTR(fw->q_d);
@@ -793,14 +817,28 @@ int forward_impl(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *W_r, c
                    slot_pos, x_perm, ws, s);
   if (rc != MOE_OK) return rc;
   if ((rc = record(ev, 3, s)) != MOE_OK) return rc;
+  GemmArgs cmb{};
+  if (fused_combine(d)) {
+    cmb.cmb_x = x;
+    cmb.cmb_perm_tok = perm_tok;
+    cmb.cmb_idx = topk_idx;
+    cmb.cmb_gate = topk_gate;
+    cmb.cmb_slot = slot_pos;
+    cmb.cmb_count = at<int>(ws, L.cmb_count);
+    cmb.cmb_y = y;
+    cmb.cmb_K = d.K;
+    cmb.cmb_N = d.N;
+    cmb.cmb_blocks = combine_blocks(d);
+  }
   rc = fw != nullptr && fp8_act(d)
            ? do_expert_ffn_e4m3(d, *di, L, x_perm, offsets, perm_gate, *fw, y_perm, ws, s, ev)
            : do_expert_ffn(d, *di, L, x_perm, offsets, perm_gate, W_g, W_u, W_d, h, y_perm, ws,
-                           s, ev, nullptr, nullptr, fw);
+                           s, ev, nullptr, nullptr, fw, fused_combine(d) ? &cmb : nullptr);
   if (rc != MOE_OK) return rc;
   if ((rc = record(ev, 5, s)) != MOE_OK) return rc;
+  // With the fused combine only tokens without an FFN slot are left (the zero-only pass).
   rc = to_status(launch_combine(x, y_perm, topk_idx, topk_gate, slot_pos, d.T, d.d, d.N, d.K,
-                                d.T * d.K, y, at<int>(ws, L.status), s));
+                                d.T * d.K, y, at<int>(ws, L.status), s, fused_combine(d)));
   if (rc != MOE_OK) return rc;
   return record(ev, 6, s);
 }
@@ -864,6 +902,7 @@ int moe_expert_ffn_fp8(const moe_dims *dims, const moe_bf16 *x_perm, const int32
                        size_t ws_bytes, void *stream) {
   MOE_REQUIRE(dims != nullptr, MOE_ERR_ARG);
   MOE_REQUIRE(dims_ok(dims) && fp8_dims_ok(*dims), MOE_ERR_SHAPE);
+  MOE_REQUIRE(!fused_combine(*dims), MOE_ERR_ARG);  // moe_forward only
   MOE_CHECK_TOKEN_PTR(x_perm, dims->T);
   MOE_CHECK_PTR(offsets);
   MOE_CHECK_TOKEN_PTR(perm_gate, dims->T);

@@ -59,6 +59,12 @@ def _full_check(w, x, wt, n_sample, seed, n_differ=8):
     st.expert_ffn()
     st.combine()
     assert torch.equal(st.y, y_fwd)
+    # The combine fused into the down projection gives the same bits.
+    fused = Stages(w, x, wt, flags=mb.FUSED_COMBINE)
+    fused.forward()
+    assert fused.device_status() == 0
+    assert torch.equal(fused.y, y_fwd), "fused combine differs at full size"
+    del fused
     # Whole-batch routing and dispatch against the oracle.
     W_r, b = wt["W_r"].cpu(), wt["b"].cpu()
     xc = x.cpu()

@@ -161,6 +161,31 @@ def test_fp8_activation_flag_layout_and_errors():
     assert lib.moe_quantize_fp8_rows(P(0x10008), 4, 128, P(0x20000), P(0x30000), None) == 3
 
 
+def test_fused_combine_flag_layout_and_errors():
+    lib = mb.lib()
+    T, d, N, Z, K, I = 64, 320, 8, 4, 3, 256
+    plain = mb.dims(T, d, N, Z, K, I)
+    dm = mb.dims(T, d, N, Z, K, I, flags=mb.FUSED_COMBINE)
+    # counters: 4 feature blocks per 256-feature m-tile of the down projection, per token
+    blocks = 4 * -(-d // 256)
+    assert mb.workspace_size(dm) == mb.workspace_size(plain) + -(-(T * blocks * 4) // 256) * 256
+    assert mb.scratch_size(dm) == mb.scratch_size(plain)
+    # every entry point other than moe_forward(_timed) refuses it (MOE_ERR_ARG) before device work
+    ws = mb.workspace_size(dm)
+    assert lib.moe_expert_ffn(ctypes.byref(dm), *[P(0x10000 * (i + 1)) for i in range(8)],
+                              P(0x1000000), ws, None) == 1
+    assert lib.moe_expert_ffn_gather(ctypes.byref(dm), *[P(0x10000 * (i + 1)) for i in range(9)],
+                                     P(0x1000000), ws, None) == 1
+    fp8 = mb.dims(T, 384, N, Z, K, I, flags=mb.FUSED_COMBINE)
+    args = [P(0x10000 * (i + 1)) for i in range(10)]
+    assert lib.moe_forward_fp8(ctypes.byref(fp8), *args, None, P(0x1000000),
+                               mb.workspace_size(fp8), None, None) == 1
+    assert lib.moe_expert_ffn_fp8(ctypes.byref(fp8), *args[:9], P(0x200000), P(0x200000),
+                                  P(0x1000000), mb.scratch_size(fp8), None) == 1
+    # moe_forward takes it, and checks the larger workspace
+    assert _fwd(dm, ws_bytes=mb.workspace_size(plain)) == 4
+
+
 def test_dense_ffn_argument_errors():
     lib = mb.lib()
     for bad in [(64, 100, 1, 0, 1, 256), (64, 128, 1, 0, 1, 96), (-1, 128, 1, 0, 1, 256)]:
@@ -178,7 +203,7 @@ def test_variant_switches_are_validated():
     lib = mb.lib()
     dm = mb.dims(64, 128, 8, 4, 3, 256, flags=mb.RENORMALIZE_GATES)
     assert mb.workspace_size(dm) == mb.workspace_size(mb.dims(64, 128, 8, 4, 3, 256))
-    assert mb.workspace_size(mb.dims(64, 128, 8, 4, 3, 256, flags=4)) == 0  # unknown flag
+    assert mb.workspace_size(mb.dims(64, 128, 8, 4, 3, 256, flags=8)) == 0  # unknown flag
     assert _fwd(mb.dims(64, 128, 8, 4, 3, 256, flags=0x80)) == 2            # MOE_ERR_SHAPE
     for gamma in (float("nan"), float("inf")):
         params = mb.PidParams(8.0, 0.1, 0.0, 0.0, gamma)
