@@ -190,7 +190,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs &a, const Tile &t,
 template <int NC>
 __device__ __forceinline__ void combine_count(const GemmArgs &a, const Tile &t, int chunks, int q,
                                               int lane, uint32_t (&fin)[NC]) {
-  __threadfence();  // this lane's y_perm stores before its arrivals
+  __threadfence();  // release: this lane's y_perm stores before its arrivals
   __syncwarp();
   const int blk = (t.m0 / (2 * kBM)) * 4 + q;
   int old[NC];
@@ -203,6 +203,7 @@ __device__ __forceinline__ void combine_count(const GemmArgs &a, const Tile &t, 
       old[c] = atomicSub(a.cmb_count + tok * a.cmb_blocks + blk, 1);
     }
   }
+  __threadfence();  // acquire: a lane that completed a count orders it before the warp's vote
 #pragma unroll
   for (int c = 0; c < NC; ++c) fin[c] = __ballot_sync(0xffffffffu, old[c] == 1);
 }
@@ -210,7 +211,7 @@ __device__ __forceinline__ void combine_count(const GemmArgs &a, const Tile &t, 
 // Sums the completed tokens' blocks of y, four tokens at a time (eight lanes, 16 bytes each).
 __device__ __forceinline__ void combine_finish(const GemmArgs &a, const Tile &t, int tok0,
                                                uint32_t fin, int q, int lane) {
-  __threadfence();  // the other tiles' rows, whose arrivals preceded ours, are visible
+  __threadfence();  // the rows of the tiles whose arrivals preceded ours, for every lane
   const int g = lane >> 3, i = lane & 7;
   const int f = t.m0 + (i < 4 ? 0 : kBM) + q * 32 + (i & 3) * 8;
   const uint16_t *y_perm = reinterpret_cast<const uint16_t *>(a.out);
