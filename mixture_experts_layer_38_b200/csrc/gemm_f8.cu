@@ -31,9 +31,10 @@
 // allocator and MMA issuer, warps 2-5 promotion and epilogue (warp w reads TMEM lane quarter
 // w mod 4), warp 6 loads each block's scales (s_x per token times s_w per sub-tile) into a
 // shared-memory slot per partial-sum buffer, up to four blocks ahead of the promotion, so the
-// promotion never waits on a global load.  Every wait is bounded; on timeout the kernel records MOE_DEV_WAIT_TIMEOUT and all
-// roles unwind (the epilogue warps agree on stopping before their shared barriers, so none is
-// left waiting at one), in-flight copies and MMAs are drained and TMEM is freed.
+// promotion never waits on a global load.  Every wait is bounded; on timeout the kernel
+// records MOE_DEV_WAIT_TIMEOUT and all roles unwind (the epilogue warps agree on stopping before
+// their shared barriers, so none is left waiting at one), in-flight copies and MMAs are drained
+// and TMEM is freed.
 #include <cuda_fp8.h>
 
 #include "device.cuh"
