@@ -11,6 +11,8 @@
 //   usage so the activated amount per token holds near a target (law: see moe_bias_update in
 //   the public header).  Optionally followed by the per-expert term of the aux-loss-free
 //   scheme the PID refines: b_i += gamma * sign(mean load - load_i), sign from integers.
+#include <algorithm>
+
 #include "device.cuh"
 #include "kernels.cuh"
 
@@ -18,6 +20,7 @@ namespace moe {
 namespace {
 
 constexpr int kCombineThreads = 128;
+constexpr int kCombineMinBlocks = 1184;  // 8 blocks per SM of a B200
 constexpr int kMaxK = 32;
 
 __global__ void __launch_bounds__(kCombineThreads)
@@ -51,7 +54,10 @@ __global__ void __launch_bounds__(kCombineThreads)
   const float zsum = s_zsum;
   const int nffn = s_nffn;
   if (zero_only && nffn > 0) return;  // written by the combine fused into the down projection
-  for (int i = threadIdx.x; i < d16; i += kCombineThreads) {
+  // Block (t, s) covers slice s of the token's row (one slice unless the batch is small).
+  const int per = (d16 + (int)gridDim.y - 1) / (int)gridDim.y;
+  const int i_end = min(d16, ((int)blockIdx.y + 1) * per);
+  for (int i = (int)blockIdx.y * per + threadIdx.x; i < i_end; i += kCombineThreads) {
     float acc[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[j] = 0.f;
@@ -117,7 +123,12 @@ cudaError_t launch_combine(const uint16_t *x, const uint16_t *y_perm, const int3
                            int K, int rows, uint16_t *y, int *status, cudaStream_t stream,
                            bool zero_only) {
   if (T == 0) return cudaSuccess;
-  combine_kernel<<<T, kCombineThreads, 0, stream>>>(
+  // Small batches: split each token's row over several blocks (at least ~1184 blocks, slices of
+  // at least 128 16-byte pieces) so the row loads of a few tokens spread over every SM.
+  const int d16 = d / 8;
+  const int max_slices = std::max(1, d16 / kCombineThreads);
+  const int slices = std::min(max_slices, std::max(1, (kCombineMinBlocks + T - 1) / T));
+  combine_kernel<<<dim3(T, slices), kCombineThreads, 0, stream>>>(
       reinterpret_cast<const uint4 *>(x), reinterpret_cast<const uint4 *>(y_perm), topk_idx,
       topk_gate, slot_pos, T, d / 8, N, K, rows, reinterpret_cast<uint4 *>(y), status,
       zero_only);
