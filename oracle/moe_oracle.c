@@ -21,11 +21,15 @@
  *     gate weights are the router's softmax outputs, not the biased scores;
  *   - a zero-computation expert returns its input unchanged;
  *   - y_t = sum over the K selected experts of g_i * E_i(x_t).
- * Readings where the pages are silent (all listed in the design notes of the repository):
+ * Readings where the pages are silent:
  *   - bias added to the softmax probability p_i (not to the logit); ties -> lower index;
- *   - gates are NOT renormalised over the selected set;
+ *   - gates are NOT renormalised over the selected set (renormalisation is an option:
+ *     oracle_renormalize_gates);
  *   - an FFN expert is SwiGLU: E(x) = W_d (silu(W_g x) * (W_u x)), silu(z) = z / (1 + e^-z);
- *   - the PID law acts on the mean number of FFN experts per token (see oracle_pid_step).
+ *   - the PID law acts on the mean number of FFN experts per token (see oracle_pid_step),
+ *     optionally followed by the per-expert balancing term (oracle_balance_step);
+ *   - FP8 (optional): E4M3 weights in 128 x 128 blocks, and optionally E4M3 activations in
+ *     1 x 128 blocks, each block with a power-of-two scale (see the FP8 section).
  *
  * Arithmetic: every floating-point step is fp64 except the PID controller, which is fp32 by
  * definition of its state; compile with -ffp-contract=off so no FMA contraction changes it.
