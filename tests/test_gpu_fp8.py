@@ -217,3 +217,36 @@ def test_forward_fp8_activations_tiny_matches_oracle():
                                 wt_deq["W_u"], wt_deq["W_d"], w.N, fp8_act=True)
     assert int(counts.sum().item()) == w.T * w.K
     assert_y_close(oracle.bf16_to_f64(to_np(y)), ref, "tiny fp8-activation forward")
+
+
+def test_fp8_activations_edge_inputs():
+    # All-zero token rows (every block scale 1, codes 0), rows scaled by 2^12 and 2^-12 (block
+    # exponents far from 0 both ways), a batch of one token, and experts left without tokens.
+    w, x, wt, fw, wt_deq = _fp8_case("tiny", T=1, seed=6)
+    for T in (1, 40):
+        w, x, wt, fw, wt_deq = _fp8_case("tiny", T=T, seed=6)
+        x = x.float()
+        if T > 1:
+            x[0] = 0
+            x[1] *= 2.0 ** 12
+            x[2] *= 2.0 ** -12
+        x = x.to(torch.bfloat16)
+        dm = mb.dims(w.T, w.d, w.N, w.Z, w.K, w.I, flags=mb.FP8_ACTIVATIONS)
+        ws = mb.alloc_workspace(dm, DEV)
+        y = torch.zeros((w.T, w.d), dtype=torch.bfloat16, device=DEV)
+        counts = torch.zeros(w.E, dtype=torch.int32, device=DEV)
+        mb.moe_forward_fp8(dm, x.to(DEV), wt["W_r"].to(DEV), wt["b"].to(DEV), fw, y, counts, ws)
+        torch.cuda.synchronize()
+        assert mb.moe_last_device_error(ws) == 0
+        r = oracle.router(x, wt["W_r"], wt["b"], w.K)
+        np.testing.assert_array_equal(to_np(counts), np.bincount(r["topk_idx"].reshape(-1),
+                                                                 minlength=w.E))
+        ref = oracle.combine_tokens(np.arange(w.T), x, r["topk_idx"], r["topk_gate"],
+                                    wt_deq["W_g"], wt_deq["W_u"], wt_deq["W_d"], w.N, fp8_act=True)
+        got = oracle.bf16_to_f64(to_np(y))
+        if T > 1:
+            assert np.all(got[0] == 0.0) and np.all(ref[0] == 0.0)
+            # each token against its own magnitude, so the 2^-12 row is checked too
+            for t in (1, 2):
+                assert_y_close(got[t:t + 1], ref[t:t + 1], f"fp8-activation token {t}")
+        assert_y_close(got, ref, f"fp8-activation edge inputs T={T}")
