@@ -255,3 +255,18 @@ def test_fp8_activations_edge_inputs():
             for t in (1, 2):
                 assert_y_close(got[t:t + 1], ref[t:t + 1], f"fp8-activation token {t}")
         assert_y_close(got, ref, f"fp8-activation edge inputs T={T}")
+
+
+def test_fp8_activations_with_renormalized_gates():
+    w, x, wt, fw, wt_deq = _fp8_case("tiny", seed=7)
+    dm = mb.dims(w.T, w.d, w.N, w.Z, w.K, w.I,
+                 flags=mb.FP8_ACTIVATIONS | mb.RENORMALIZE_GATES)
+    ws = mb.alloc_workspace(dm, DEV)
+    y = torch.zeros((w.T, w.d), dtype=torch.bfloat16, device=DEV)
+    mb.moe_forward_fp8(dm, x.to(DEV), wt["W_r"].to(DEV), wt["b"].to(DEV), fw, y, None, ws)
+    torch.cuda.synchronize()
+    assert mb.moe_last_device_error(ws) == 0
+    r = oracle.router(x, wt["W_r"], wt["b"], w.K, renormalize=True)
+    ref = oracle.combine_tokens(np.arange(w.T), x, r["topk_idx"], r["topk_gate"], wt_deq["W_g"],
+                                wt_deq["W_u"], wt_deq["W_d"], w.N, fp8_act=True)
+    assert_y_close(oracle.bf16_to_f64(to_np(y)), ref, "tiny fp8-activation renormalised")

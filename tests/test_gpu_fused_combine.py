@@ -93,3 +93,16 @@ def test_fused_combine_zero_tokens():
     y = torch.empty((0, w.d), dtype=torch.bfloat16, device="cuda")
     mb.moe_forward(dm, x, g["W_r"], g["b"], g["W_g"], g["W_u"], g["W_d"], y, None, ws)
     assert mb.moe_last_device_error(ws) == 0
+
+
+def test_fused_combine_with_renormalized_gates():
+    # The flags combine: renormalised gates change topk_gate, which the fused epilogue reads
+    # for the zero-expert term and the combine pass uses alike.
+    w, x, wt = _case(WORKLOADS["mid"], T=500, seed=5)
+    plain = Stages(w, x, wt, flags=mb.RENORMALIZE_GATES)
+    plain.forward()
+    fused = Stages(w, x, wt, flags=mb.RENORMALIZE_GATES | mb.FUSED_COMBINE)
+    fused.forward()
+    torch.cuda.synchronize()
+    assert plain.device_status() == 0 and fused.device_status() == 0
+    assert torch.equal(plain.y, fused.y)
