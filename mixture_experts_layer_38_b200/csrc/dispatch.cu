@@ -116,6 +116,78 @@ __global__ void __launch_bounds__(kDispatchChunk)
   }
 }
 
+// A batch of one chunk (T <= 256): histogram, scans and permutation in one block -- the same
+// masks, the same ranks and the same tables as the three kernels above, without their two
+// extra launches and second mask build (decode-sized batches are launch- and latency-bound).
+// Thread i owns experts [i * P, i * P + P), P = ceil(E / 256), so the exclusive scan over
+// experts is a block scan of per-thread sums.
+__global__ void __launch_bounds__(kDispatchChunk)
+    dispatch_small_kernel(const int32_t *__restrict__ topk_idx,
+                          const float *__restrict__ topk_gate, int T, int K, int N, int E,
+                          int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
+                          int32_t *__restrict__ perm_tok, float *__restrict__ perm_gate,
+                          int32_t *__restrict__ slot_pos, int *status) {
+  extern __shared__ uint32_t masks[];  // [kWarps * E] masks, then [E] first rows
+  int *first = reinterpret_cast<int *>(masks + kWarps * E);
+  __shared__ int warp_tot[kWarps];
+  build_masks(topk_idx, T, K, E, masks, status);
+  const int P = (E + kDispatchChunk - 1) / kDispatchChunk;  // <= 4
+  const int e0 = threadIdx.x * P;
+  int c[4];
+  int mine = 0;  // this thread's FFN rows, in expert order
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    c[j] = 0;
+    const int e = e0 + j;
+    if (j < P && e < E) {
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) c[j] += __popc(masks[w * E + e]);
+      counts[e] = c[j];
+      if (e < N) mine += c[j];
+    }
+  }
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  int incl = mine;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  if (lane == 31) warp_tot[wid] = incl;
+  __syncthreads();
+  int run = incl - mine;
+  for (int w = 0; w < wid; ++w) run += warp_tot[w];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int e = e0 + j;
+    if (j < P && e < N) {
+      first[e] = run;
+      run += c[j];
+      offsets[e + 1] = run;
+    }
+  }
+  if (threadIdx.x == 0) offsets[0] = 0;
+  __syncthreads();
+  const int t = threadIdx.x;
+  if (t >= T) return;
+  const uint32_t lower = (1u << lane) - 1u;
+  for (int k = 0; k < K; ++k) {
+    const long long slot = (long long)t * K + k;
+    const int e = __ldg(topk_idx + slot);
+    if (e < 0 || e >= N) {  // zero expert (or an invalid id, already flagged)
+      slot_pos[slot] = -1;
+      continue;
+    }
+    int rank = 0;
+    for (int w2 = 0; w2 < wid; ++w2) rank += __popc(masks[w2 * E + e]);
+    rank += __popc(masks[wid * E + e] & lower);
+    const int r = first[e] + rank;
+    perm_tok[r] = t;
+    perm_gate[r] = __ldg(topk_gate + slot);
+    slot_pos[slot] = r;
+  }
+}
+
 // x_perm[r] = x[perm_tok[r]] for r < A = offsets[N]; one warp per row, 16-byte accesses.
 __global__ void __launch_bounds__(256)
     gather_rows_kernel(const uint4 *__restrict__ x, int d16, int T,
@@ -153,6 +225,15 @@ cudaError_t launch_dispatch(const uint16_t *x, const int32_t *topk_idx, const fl
                             int num_sms, cudaStream_t stream) {
   const int nchunks = dispatch_chunks(T);
   const size_t mask_bytes = sizeof(uint32_t) * kWarps * E;
+  if (nchunks == 1) {  // one block does the histogram, the scans and the permutation
+    dispatch_small_kernel<<<1, kDispatchChunk, mask_bytes + sizeof(int) * E, stream>>>(
+        topk_idx, topk_gate, T, K, N, E, counts, offsets, perm_tok, perm_gate, slot_pos, status);
+    if (x_perm != nullptr)
+      gather_rows_kernel<<<num_sms * 8, 256, 0, stream>>>(
+          reinterpret_cast<const uint4 *>(x), d / 8, T, perm_tok, offsets + N,
+          reinterpret_cast<uint4 *>(x_perm), status);
+    return cudaGetLastError();
+  }
   if (nchunks > 0) {
     dispatch_hist_kernel<<<nchunks, kDispatchChunk, mask_bytes, stream>>>(topk_idx, T, K, E,
                                                                           chunk_counts, status);
