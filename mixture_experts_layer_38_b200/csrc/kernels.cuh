@@ -116,8 +116,12 @@ cudaError_t launch_quantize_fp8(const uint16_t *w, long long G, long long R, lon
 // FP8 activations: rows of the bf16 matrix x [R, C] (C a multiple of 128) -> E4M3 codes q
 // [R, C] and one power-of-two scale per 1 x 128 block, stored block-major:
 // scale_t[(c / 128) * R + r].  Rows from *live_rows on are skipped (live_rows may be NULL).
+// With row_index, output row r quantises row row_index[r] of x ([src_rows, C]); indices outside
+// that range are reported (MOE_DEV_BAD_ROWS on status) and their rows skipped.
 cudaError_t launch_quantize_fp8_rows(const uint16_t *x, long long R, int C, const int *live_rows,
-                                     uint8_t *q, float *scale_t, cudaStream_t stream);
+                                     uint8_t *q, float *scale_t, cudaStream_t stream,
+                                     const int32_t *row_index = nullptr, long long src_rows = 0,
+                                     int *status = nullptr);
 
 // ------------------------------------------------------------------ routing
 // logits [splits][T][E] fp32 -> softmax, biased top-K, ascending ids.

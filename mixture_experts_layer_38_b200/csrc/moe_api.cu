@@ -443,10 +443,12 @@ int do_expert_ffn(const moe_dims &d, const DeviceInfo &di, const Layout &L,
 // The expert FFN with FP8 weights and FP8 activations: x_perm's rows are quantised (1 x 128
 // blocks) into the workspace, the up-projection reads the codes on the tensor cores and writes
 // h as codes and scales, and the down projection reads those.
+// x_perm NULL: the token rows are quantised straight from x through perm_tok (no bf16 copy).
 int do_expert_ffn_e4m3(const moe_dims &d, const DeviceInfo &di, const Layout &L,
                        const moe_bf16 *x_perm, const int32_t *offsets, const float *perm_gate,
                        const Fp8Weights &fw, moe_bf16 *y_perm, void *ws, cudaStream_t stream,
-                       void *const *events = nullptr) {
+                       void *const *events = nullptr, const moe_bf16 *x = nullptr,
+                       const int32_t *perm_tok = nullptr) {
   if (d.T == 0 || d.N == 0) return record(events, 4, stream);
   const uint64_t rows = (uint64_t)d.T * d.K;
   int *status = at<int>(ws, L.status);
@@ -455,9 +457,12 @@ int do_expert_ffn_e4m3(const moe_dims &d, const DeviceInfo &di, const Layout &L,
   uint8_t *hq = at<uint8_t>(ws, L.hq);
   float *sh = at<float>(ws, L.sh);
   // Only the rows of the FFN experts' groups (offsets[N] of them) are quantised.
-  if (launch_quantize_fp8_rows(x_perm, (long long)rows, d.d, offsets + d.N, xq, sx, stream) !=
-      cudaSuccess)
-    return MOE_ERR_CUDA;
+  const cudaError_t qe =
+      x_perm != nullptr
+          ? launch_quantize_fp8_rows(x_perm, (long long)rows, d.d, offsets + d.N, xq, sx, stream)
+          : launch_quantize_fp8_rows(x, (long long)rows, d.d, offsets + d.N, xq, sx, stream,
+                                     perm_tok, d.T, status);
+  if (qe != cudaSuccess) return MOE_ERR_CUDA;
   GemmArgs up{};
   bool ok = make_map_e4m3(&up.map_a0, fw.q_g, (uint64_t)d.N * d.I, (uint64_t)d.d, 128) &&
             make_map_e4m3(&up.map_a1, fw.q_u, (uint64_t)d.N * d.I, (uint64_t)d.d, 128);
@@ -813,8 +818,10 @@ int forward_impl(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *W_r, c
   if ((rc = record(ev, 2, s)) != MOE_OK) return rc;
   // The gathered copy x_perm and tiled token loads: faster at large T than gathering rows
   // inside the up-projection (moe_expert_ffn_gather), whose row-by-row copies cost more.
+  // With FP8 activations the up-projection's quantiser reads the token rows from x itself.
+  const bool fp8_rows = fw != nullptr && fp8_act(d);
   rc = do_dispatch(d, *di, L, x, topk_idx, topk_gate, cnt, offsets, perm_tok, perm_gate,
-                   slot_pos, x_perm, ws, s);
+                   slot_pos, fp8_rows ? nullptr : x_perm, ws, s);
   if (rc != MOE_OK) return rc;
   if ((rc = record(ev, 3, s)) != MOE_OK) return rc;
   GemmArgs cmb{};
@@ -830,8 +837,9 @@ int forward_impl(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *W_r, c
     cmb.cmb_N = d.N;
     cmb.cmb_blocks = combine_blocks(d);
   }
-  rc = fw != nullptr && fp8_act(d)
-           ? do_expert_ffn_e4m3(d, *di, L, x_perm, offsets, perm_gate, *fw, y_perm, ws, s, ev)
+  rc = fp8_rows
+           ? do_expert_ffn_e4m3(d, *di, L, nullptr, offsets, perm_gate, *fw, y_perm, ws, s, ev,
+                                x, perm_tok)
            : do_expert_ffn(d, *di, L, x_perm, offsets, perm_gate, W_g, W_u, W_d, h, y_perm, ws,
                            s, ev, nullptr, nullptr, fw, fused_combine(d) ? &cmb : nullptr);
   if (rc != MOE_OK) return rc;

@@ -73,13 +73,16 @@ __global__ void __launch_bounds__(kQuantThreads)
 // FP8 activations: one scale per 1 x 128 block of a row, by the same rule.  One warp per row
 // and pair of blocks: lanes 0-15 take block 2p, lanes 16-31 block 2p + 1, eight values (16
 // bytes) per lane, so each half-warp reads one 256-byte block segment.  Rows from *live_rows on
-// (when given) are skipped: grouped rows past the last expert's hold nothing.
+// (when given) are skipped: grouped rows past the last expert's hold nothing.  With row_index,
+// output row r is the quantised row row_index[r] of x (src_rows rows): the dispatch gather and
+// the quantisation in one pass; an index outside [0, src_rows) is reported and its row skipped.
 constexpr int kRowQuantThreads = 256;
 
 __global__ void __launch_bounds__(kRowQuantThreads)
     quantize_rows_fp8_kernel(const uint16_t *__restrict__ x, long long R, int C,
-                             const int *__restrict__ live_rows, uint8_t *__restrict__ q,
-                             float *__restrict__ scale_t) {
+                             const int *__restrict__ live_rows,
+                             const int32_t *__restrict__ row_index, long long src_rows,
+                             uint8_t *__restrict__ q, float *__restrict__ scale_t, int *status) {
   const int lane = threadIdx.x & 31;
   const int CB = C / 128, pairs = (CB + 1) / 2;
   const long long gw = (long long)blockIdx.x * (kRowQuantThreads / 32) + (threadIdx.x >> 5);
@@ -88,10 +91,19 @@ __global__ void __launch_bounds__(kRowQuantThreads)
   long long rows = R;
   if (live_rows != nullptr) rows = min(rows, (long long)max(__ldg(live_rows), 0));
   if (r >= rows) return;  // uniform over the warp
+  long long src = r;
+  if (row_index != nullptr) {
+    src = __ldg(row_index + r);
+    if (src < 0 || src >= src_rows) {
+      if (lane == 0) record_status(status, MOE_DEV_BAD_ROWS);
+      return;
+    }
+  }
   const bool active = cb < CB;
-  const long long off = r * C + (long long)cb * 128 + (lane & 15) * 8;
+  const long long col = (long long)cb * 128 + (lane & 15) * 8;
+  const long long off = r * C + col;
   uint4 v = make_uint4(0u, 0u, 0u, 0u);
-  if (active) v = *reinterpret_cast<const uint4 *>(x + off);
+  if (active) v = *reinterpret_cast<const uint4 *>(x + src * C + col);
   const uint32_t u[4] = {v.x, v.y, v.z, v.w};
   float amax = 0.f;
 #pragma unroll
@@ -120,13 +132,14 @@ __global__ void __launch_bounds__(kRowQuantThreads)
 }  // namespace
 
 cudaError_t launch_quantize_fp8_rows(const uint16_t *x, long long R, int C, const int *live_rows,
-                                     uint8_t *q, float *scale_t, cudaStream_t stream) {
+                                     uint8_t *q, float *scale_t, cudaStream_t stream,
+                                     const int32_t *row_index, long long src_rows, int *status) {
   if (R == 0 || C == 0) return cudaSuccess;
   const long long warps = R * ((C / 128 + 1) / 2);
   const long long blocks = (warps + kRowQuantThreads / 32 - 1) / (kRowQuantThreads / 32);
   if (blocks > 0x7fffffffll) return cudaErrorInvalidValue;
-  quantize_rows_fp8_kernel<<<(unsigned)blocks, kRowQuantThreads, 0, stream>>>(x, R, C, live_rows,
-                                                                           q, scale_t);
+  quantize_rows_fp8_kernel<<<(unsigned)blocks, kRowQuantThreads, 0, stream>>>(
+      x, R, C, live_rows, row_index, src_rows, q, scale_t, status);
   return cudaGetLastError();
 }
 
