@@ -261,6 +261,12 @@ def test_work_model_per_unit_figures():
                       "dispatch": 160, "combine": 208}
     _, _, _, nbytes8 = _bench().work_model(w, [3, 0, 2, 3], wb=1)  # E4M3 weight codes
     assert nbytes8["ffn_up_gemm"] == 512 + 80 + 160 and nbytes8["ffn_down_gemm"] == 256 + 240
+    # FP8 activations: one byte per x_perm and h element in the GEMMs, plus the up stage's row
+    # quantiser (2 bytes read + 1 written per element of the A x d token rows); y_perm stays bf16
+    _, _, flops8a, nbytes8a = _bench().work_model(w, [3, 0, 2, 3], wb=1, ab=1)
+    assert flops8a == flops
+    assert nbytes8a["ffn_up_gemm"] == 512 + 40 + 80 + 120
+    assert nbytes8a["ffn_down_gemm"] == 256 + 80 + 80
 
 
 def test_gemm_source_hash_ignores_comments_only():
