@@ -234,7 +234,7 @@ def work_model(w, counts, wb=2, ab=2):
         "ffn_up_gemm": U * 2 * I * d * wb + A * d * ab + A * I * ab +
                        (A * d * 3 if ab == 1 else 0),
         "ffn_down_gemm": U * d * I * wb + A * I * ab + A * d * 2,
-        "dispatch": 2 * A * d * 2,
+        "dispatch": (T + A) * d * 2,  # each token row read once, each slot row written
         "combine": (A + 2 * T) * d * 2,
     }
     return A, U, flops, bytes_

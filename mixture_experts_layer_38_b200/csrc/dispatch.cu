@@ -1,5 +1,5 @@
 // dispatch.cu -- group the FFN slots by expert: deterministic histogram, exclusive scans and a
-// stable token permutation, then a 16-byte-vectorised gather of the token rows.
+// stable token permutation, then a 16-byte-vectorised copy of each token row to its slots.
 //
 // Zero-computation experts return their input ("衝上熱搜！美團大模型，靠「快」火了", §零計算專家), so
 // only slots whose expert id is < N are grouped and copied; zero-expert slots are counted (for
@@ -10,7 +10,8 @@
 // atomicOr (the final mask does not depend on timing), so the rank of a slot among the same
 // expert's slots is: slots in earlier chunks (column scan of the per-chunk histogram) + slots in
 // earlier warps of the chunk (popcounts) + earlier lanes of the warp (popcount of the lower mask
-// bits).  No float atomics, no spin waits: four plain kernels.
+// bits).  No float atomics, no spin waits: four plain kernels (one block for the tables when
+// the batch is a single chunk), the last copying each token's row to its slots' rows.
 #include "device.cuh"
 #include "kernels.cuh"
 
@@ -188,7 +189,53 @@ __global__ void __launch_bounds__(kDispatchChunk)
   }
 }
 
-// x_perm[r] = x[perm_tok[r]] for r < A = offsets[N]; one warp per row, 16-byte accesses.
+// x_perm[slot_pos[t, k]] = x[t] for every FFN slot (t, k): one warp per token reads the token's
+// row once and writes it to each of its FFN slots' rows (16-byte accesses, four in flight per
+// lane).  Token-major on purpose: a gather over the grouped rows visits a token once per slot,
+// in expert order, and when x exceeds the L2 (prefill: 201 MB) each visit is a DRAM read; with
+// x in the L2, the gather below has the parallelism (a warp per row, not per token).
+constexpr int kScatterWarps = 8;
+
+__global__ void __launch_bounds__(32 * kScatterWarps)
+    scatter_rows_kernel(const uint4 *__restrict__ x, int d16, int T, int K,
+                        const int32_t *__restrict__ slot_pos, int rows,
+                        uint4 *__restrict__ x_perm, int *status) {
+  __shared__ int dst_row[kScatterWarps][32];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warps = gridDim.x * kScatterWarps;
+  for (int t = blockIdx.x * kScatterWarps + w; t < T; t += warps) {
+    int r = -1;
+    if (lane < K) {
+      r = __ldg(slot_pos + (long long)t * K + lane);
+      if (r < -1 || r >= rows) {  // -1: a zero-expert slot
+        record_status(status, MOE_DEV_BAD_ROWS);
+        r = -1;
+      }
+    }
+    const uint32_t slots = __ballot_sync(0xffffffffu, r >= 0);
+    dst_row[w][lane] = r;
+    __syncwarp();
+    if (slots != 0u) {
+      const uint4 *src = x + (long long)t * d16;
+      for (int i0 = lane; i0 < d16; i0 += 128) {
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (i0 + 32 * u < d16) v[u] = __ldg(src + i0 + 32 * u);
+        for (uint32_t m = slots; m != 0u; m &= m - 1) {
+          uint4 *dst = x_perm + (long long)dst_row[w][__ffs(m) - 1] * d16;
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (i0 + 32 * u < d16) dst[i0 + 32 * u] = v[u];
+        }
+      }
+    }
+    __syncwarp();
+  }
+}
+
+// x_perm[r] = x[perm_tok[r]] for r < A = offsets[N]; one warp per row, 16-byte accesses: more
+// warps than tokens, the better choice while x stays in the L2 (decode, mid).
 __global__ void __launch_bounds__(256)
     gather_rows_kernel(const uint4 *__restrict__ x, int d16, int T,
                        const int32_t *__restrict__ perm_tok, const int32_t *__restrict__ a_rows,
@@ -216,6 +263,23 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// Token rows of at least this many bytes in all (about half the L2) are copied token-major.
+constexpr long long kScatterMinBytes = 64ll << 20;
+
+cudaError_t copy_rows(const uint16_t *x, int T, int d, int K, int N, const int32_t *perm_tok,
+                      const int32_t *offsets, const int32_t *slot_pos, uint16_t *x_perm,
+                      int *status, int num_sms, cudaStream_t stream) {
+  if ((long long)T * d * 2 >= kScatterMinBytes)
+    scatter_rows_kernel<<<num_sms * 8, 32 * kScatterWarps, 0, stream>>>(
+        reinterpret_cast<const uint4 *>(x), d / 8, T, K, slot_pos, T * K,
+        reinterpret_cast<uint4 *>(x_perm), status);
+  else
+    gather_rows_kernel<<<num_sms * 8, 256, 0, stream>>>(
+        reinterpret_cast<const uint4 *>(x), d / 8, T, perm_tok, offsets + N,
+        reinterpret_cast<uint4 *>(x_perm), status);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_dispatch(const uint16_t *x, const int32_t *topk_idx, const float *topk_gate,
@@ -229,9 +293,8 @@ cudaError_t launch_dispatch(const uint16_t *x, const int32_t *topk_idx, const fl
     dispatch_small_kernel<<<1, kDispatchChunk, mask_bytes + sizeof(int) * E, stream>>>(
         topk_idx, topk_gate, T, K, N, E, counts, offsets, perm_tok, perm_gate, slot_pos, status);
     if (x_perm != nullptr)
-      gather_rows_kernel<<<num_sms * 8, 256, 0, stream>>>(
-          reinterpret_cast<const uint4 *>(x), d / 8, T, perm_tok, offsets + N,
-          reinterpret_cast<uint4 *>(x_perm), status);
+      return copy_rows(x, T, d, K, N, perm_tok, offsets, slot_pos, x_perm, status, num_sms,
+                       stream);
     return cudaGetLastError();
   }
   if (nchunks > 0) {
@@ -244,9 +307,8 @@ cudaError_t launch_dispatch(const uint16_t *x, const int32_t *topk_idx, const fl
         topk_idx, topk_gate, T, K, N, E, chunk_counts, offsets, perm_tok, perm_gate, slot_pos,
         status);
     if (x_perm != nullptr)  // NULL: the up-projection gathers the rows itself
-      gather_rows_kernel<<<num_sms * 8, 256, 0, stream>>>(
-          reinterpret_cast<const uint4 *>(x), d / 8, T, perm_tok, offsets + N,
-          reinterpret_cast<uint4 *>(x_perm), status);
+      return copy_rows(x, T, d, K, N, perm_tok, offsets, slot_pos, x_perm, status, num_sms,
+                       stream);
   }
   return cudaGetLastError();
 }

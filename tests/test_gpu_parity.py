@@ -180,6 +180,36 @@ def test_expert_ffn_gather_matches_oracle_and_unfused(name, T):
     assert_y_close(oracle.bf16_to_f64(to_np(st.y_perm)[:A]), rows, f"{name} gathered y_perm")
 
 
+def test_dispatch_row_copy_token_major():
+    # Token rows of 64 MB or more are copied token-major (each x row read once, written to its
+    # slots' rows); the grouped rows must equal x[perm_tok] exactly, as with the row gather.
+    w = Workload("wide", T=8192, d=4096, N=8, Z=4, K=3, I=256)
+    g = torch.Generator(device=DEV).manual_seed(9)
+    x = torch.randn((w.T, w.d), generator=g, device=DEV).to(torch.bfloat16)
+    W_r = (torch.randn((w.E, w.d), generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    b = torch.zeros(w.E, device=DEV)
+    dm = mb.dims(w.T, w.d, w.N, w.Z, w.K, w.I)
+    ws = mb.alloc_workspace(dm, DEV, scratch_only=True)
+    R = w.T * w.K
+    i32 = dict(dtype=torch.int32, device=DEV)
+    idx, gate = torch.empty((w.T, w.K), **i32), torch.empty((w.T, w.K), dtype=torch.float32,
+                                                            device=DEV)
+    mb.moe_route(dm, x, W_r, b, idx, gate, None, ws)
+    counts, offsets = torch.empty(w.E, **i32), torch.empty(w.N + 1, **i32)
+    perm_tok, slot_pos = torch.empty(R, **i32), torch.empty((w.T, w.K), **i32)
+    perm_gate = torch.empty(R, dtype=torch.float32, device=DEV)
+    x_perm = torch.zeros((R, w.d), dtype=torch.bfloat16, device=DEV)
+    mb.moe_dispatch(dm, x, idx, gate, counts, offsets, perm_tok, perm_gate, slot_pos, x_perm, ws)
+    torch.cuda.synchronize()
+    assert mb.moe_last_device_error(ws) == 0
+    A = int(offsets[-1].item())
+    assert A > 0
+    assert torch.equal(x_perm[:A], x[perm_tok[:A].long()])
+    assert (x_perm[A:] == 0).all()  # rows past the groups are not written
+    check_dispatch_vs_oracle(to_np(idx), to_np(gate), to_np(counts), to_np(offsets),
+                             to_np(perm_tok), to_np(perm_gate), to_np(slot_pos), w.N, w.E)
+
+
 def test_dispatch_without_gather_leaves_x_perm_alone():
     w, x, wt = _case(WORKLOADS["tiny"])
     st = Stages(w, x, wt)

@@ -258,7 +258,7 @@ def test_work_model_per_unit_figures():
     assert (A, U) == (5, 2)
     assert flops == {"router_gemm": 256, "ffn_up_gemm": 2560, "ffn_down_gemm": 1280}
     assert nbytes == {"router_gemm": 192, "ffn_up_gemm": 1264, "ffn_down_gemm": 752,
-                      "dispatch": 160, "combine": 208}
+                      "dispatch": 144, "combine": 208}
     _, _, _, nbytes8 = _bench().work_model(w, [3, 0, 2, 3], wb=1)  # E4M3 weight codes
     assert nbytes8["ffn_up_gemm"] == 512 + 80 + 160 and nbytes8["ffn_down_gemm"] == 256 + 240
     # FP8 activations: one byte per x_perm and h element in the GEMMs, plus the up stage's row
