@@ -49,9 +49,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # while the kernel and its launch set-up are unchanged (sha1 of the code, comments removed, of
 # the GEMM kernel and of the file that builds its tensor maps, at capture time).
 NCU_TRAFFIC = {
-    ("prefill", "ffn_up_gemm"): {"bytes_per_launch": 41377593600, "src": "5a35ac00afb5"},
-    ("prefill", "ffn_down_gemm"): {"bytes_per_launch": 17432248064, "src": "5a35ac00afb5"},
-    ("decode", "ffn_up_gemm"): {"bytes_per_launch": 7316193024, "src": "5a35ac00afb5"},
+    # DRAM bytes per launch of the dominant kernel (dram__bytes_read.sum + dram__bytes_write.sum)
+    # for the sources hashing to "src".  Decode streams each used expert's weights once, so the
+    # figures come from a decode-shaped capture with 128 experts (102 used) scaled to the decode
+    # workload's 145 used experts (the decode-shaped DRAM summary under profiles/); prefill's
+    # traffic does not scale that way and was not captured at full size for this build (null).
+    ("decode", "ffn_up_gemm"): {"bytes_per_launch": 7315470758, "src": "869fc7a06349"},
+    ("decode+fp8+act", "ffn_up_gemm"): {"bytes_per_launch": 3779534105, "src": "869fc7a06349"},
 }
 
 
