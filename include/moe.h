@@ -120,7 +120,10 @@ const char *moe_strerror(int code);
 /* Workspace bytes needed by moe_forward for these dims (0 for invalid dims).  The workspace
  * holds the status word, router logits, top-K results, dispatch tables, the grouped
  * activations x_perm [T*K, d], the SwiGLU activations h [T*K, I] and the expert outputs
- * y_perm [T*K, d]; about (2d + I) * 2 * T * K bytes plus small tables. */
+ * y_perm [T*K, d]; about (2d + I) * 2 * T * K bytes plus small tables.  The flags add their
+ * regions: MOE_FP8_ACTIVATIONS the codes and block scales of the token rows and of h (in the
+ * scratch part, about (d + I) * 1.03 * T * K bytes), MOE_FUSED_COMBINE one counter per token
+ * and 64-feature block (T * 4 * ceil(d / 256) * 4 bytes). */
 size_t moe_workspace_size(const moe_dims *dims);
 
 /* Scratch bytes needed by the staged calls (moe_route, moe_dispatch, moe_expert_ffn): the
@@ -321,7 +324,9 @@ int moe_expert_ffn_fp8(const moe_dims *dims, const moe_bf16 *x_perm, const int32
                        size_t ws_bytes, void *stream);
 
 /* moe_forward with block-quantised expert weights (the router weights stay bf16);
- * stage_events as in moe_forward_timed, or NULL. */
+ * stage_events as in moe_forward_timed, or NULL.  With MOE_FP8_ACTIVATIONS the token rows are
+ * quantised straight from x through the dispatch permutation (no bf16 copy of them is made) and
+ * both expert GEMMs multiply E4M3 by E4M3; the workspace is moe_workspace_size of those dims. */
 int moe_forward_fp8(const moe_dims *dims, const moe_bf16 *x, const moe_bf16 *W_r,
                     const float *b, const uint8_t *q_g, const float *s_g, const uint8_t *q_u,
                     const float *s_u, const uint8_t *q_d, const float *s_d, moe_bf16 *y,
